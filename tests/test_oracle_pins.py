@@ -1,0 +1,378 @@
+"""Pins for the fp64 oracle: values it must reproduce that do not come from itself.
+
+Each pin is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a wrong branch block, a wrong
+softmax normalisation) fails at least one of them; ``test_planted_mistakes``
+plants such slips in the oracle and checks that they are caught.
+"""
+import cmath
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import mla_oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def _ev(x):
+    return float(eval(x, {"math": math})) if isinstance(x, str) else float(x)
+
+
+def _evm(a):
+    return np.array([[_ev(v) for v in row] for row in a], dtype=np.float64) if isinstance(a[0], list) \
+        else np.array([_ev(v) for v in a], dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# independent brute force: pure-Python loops, RoPE as complex multiplication
+# ---------------------------------------------------------------------------
+
+def brute_rope(vec, pos, base):
+    d = len(vec)
+    out = []
+    for i in range(d // 2):
+        z = complex(vec[2 * i], vec[2 * i + 1]) * cmath.exp(1j * pos * base ** (-2.0 * i / d))
+        out += [z.real, z.imag]
+    return out
+
+
+def brute_decode_one(qn, qr, qpos, Wk, Wv, C, Kraw, n_branch, bscale, scale, base):
+    L = len(C)
+    d_c = len(C[0]) if L else len(Wv)
+    d_h, d_v = len(qn), len(Wv[0])
+    out = [0.0] * d_v
+    if L == 0:
+        return out
+    d_cb = d_c // n_branch
+    q_rot = brute_rope(qr, qpos, base)
+    for br in range(n_branch):
+        cols = range(br * d_cb, (br + 1) * d_cb)
+        logits = []
+        for t in range(L):
+            kt = brute_rope(Kraw[t], t, base)
+            content = 0.0
+            for j in range(d_h):
+                key_j = sum(C[t][c] * Wk[j][c] for c in cols)
+                content += qn[j] * key_j
+            rope_s = sum(q_rot[i] * kt[i] for i in range(len(kt)))
+            logits.append(scale * (content + rope_s))
+        mx = max(logits)
+        e = [math.exp(s - mx) for s in logits]
+        z = sum(e)
+        for t in range(L):
+            p = e[t] / z
+            for v in range(d_v):
+                val = sum(C[t][c] * Wv[c][v] for c in cols)
+                out[v] += bscale * p * val
+    return out
+
+
+def _rand_case(rng, B=2, H=2, d_h=4, d_c=8, d_v=3, d_r=4, n_branch=1, lens=(3, 5), page_size=2,
+               branch_scale=1.0, permute=True):
+    lens = np.array(lens[:B])
+    npages = (lens + page_size - 1) // page_size
+    maxp = int(npages.max())
+    P = int(npages.sum()) + 3
+    order = rng.permutation(P) if permute else np.arange(P)
+    pt = np.full((B, maxp), -1, dtype=np.int64)
+    o = 0
+    for b in range(B):
+        pt[b, :npages[b]] = order[o:o + npages[b]]
+        o += npages[b]
+    T = int(lens.sum())
+    tok_seq = np.repeat(np.arange(B), lens)
+    tok_pos = np.concatenate([np.arange(L) for L in lens]) if T else np.zeros(0, np.int64)
+    return dict(
+        q_nope=rng.standard_normal((B, H, d_h)), q_rope=rng.standard_normal((B, H, d_r)),
+        q_pos=lens.astype(np.float64) + rng.integers(0, 3, B),
+        W_UK=rng.standard_normal((H, d_h, d_c)) / np.sqrt(d_c),
+        W_UV=rng.standard_normal((H, d_c, d_v)) / np.sqrt(d_c),
+        c_kv=rng.standard_normal((T, d_c)), k_rope=rng.standard_normal((T, d_r)),
+        tok_seq=tok_seq, tok_pos=tok_pos, page_table=pt, num_pages=P, seq_lens=lens,
+        n_branch=n_branch, branch_scale=branch_scale, softmax_scale=None, rope_base=10000.0,
+    ), page_size
+
+
+def _brute_all(inp, page_size):
+    B, H = inp["q_nope"].shape[:2]
+    d_h, d_r = inp["q_nope"].shape[2], inp["q_rope"].shape[2]
+    scale = 1.0 / math.sqrt(d_h + d_r)
+    res = {}
+    for b in range(B):
+        L = int(inp["seq_lens"][b])
+        # logical token order: token t of sequence b is the packed row with tok_seq=b, tok_pos=t
+        rows = [i for i in range(len(inp["tok_seq"])) if inp["tok_seq"][i] == b]
+        rows.sort(key=lambda i: inp["tok_pos"][i])
+        C = [list(inp["c_kv"][i]) for i in rows][:L]
+        K = [list(inp["k_rope"][i]) for i in rows][:L]
+        for h in range(H):
+            res[(b, h)] = np.array(brute_decode_one(
+                list(inp["q_nope"][b, h]), list(inp["q_rope"][b, h]), float(inp["q_pos"][b]),
+                inp["W_UK"][h].tolist(), inp["W_UV"][h].tolist(), C, K,
+                inp["n_branch"], inp["branch_scale"], scale, inp["rope_base"]))
+    return res
+
+
+def _max_err(a, b):
+    return max(float(np.max(np.abs(a[k] - b[k]))) for k in a)
+
+
+@pytest.mark.parametrize("n_branch,bscale", [(1, 1.0), (2, 0.7), (4, 0.5)])
+def test_brute_force_tiny(n_branch, bscale):
+    rng = np.random.default_rng(100 + n_branch)
+    inp, ps = _rand_case(rng, n_branch=n_branch, branch_scale=bscale)
+    got = oracle.decode(inp, page_size=ps)
+    ref = _brute_all(inp, ps)
+    assert _max_err(got, ref) <= 1e-12
+
+
+def test_brute_force_empty_and_single():
+    rng = np.random.default_rng(7)
+    inp, ps = _rand_case(rng, lens=(0, 1))
+    got = oracle.decode(inp, page_size=ps)
+    ref = _brute_all(inp, ps)
+    assert _max_err(got, ref) <= 1e-12
+    assert np.all(got[(0, 0)] == 0.0) and np.all(got[(0, 1)] == 0.0)
+
+
+# ---------------------------------------------------------------------------
+# closed-form worked examples
+# ---------------------------------------------------------------------------
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden()["cases"], ids=lambda c: c["name"])
+def test_golden_worked_example(case):
+    C = _evm(case["c_kv"])
+    K = _evm(case["k_rope"])
+    out = oracle.attend_sequence(
+        _evm(case["q_nope"]), _evm(case["q_rope"]), float(case["q_pos"]),
+        np.array(case["W_UK"], dtype=np.float64), np.array(case["W_UV"], dtype=np.float64),
+        C, K, [0], n_branch=case["n_branch"], branch_scale=case["branch_scale"])
+    exp = _evm(case["expected"])
+    np.testing.assert_allclose(out, exp, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("case", _golden()["rope_cases"], ids=lambda c: c["name"])
+def test_golden_rope(case):
+    out = oracle.rope(np.array(case["x"]), float(case["pos"]), case["base"])
+    np.testing.assert_allclose(out, _evm(case["expected"]), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# RoPE invariants
+# ---------------------------------------------------------------------------
+
+def test_rope_matches_complex_multiplication():
+    rng = np.random.default_rng(3)
+    for d in (2, 4, 16, 64):
+        x = rng.standard_normal(d)
+        for pos in (0, 1, 17, 4096, 131072):
+            np.testing.assert_allclose(oracle.rope(x, pos), brute_rope(list(x), pos, 10000.0),
+                                       rtol=0, atol=1e-11)
+
+
+def test_rope_preserves_norm_and_is_relative():
+    rng = np.random.default_rng(4)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for pos in (0, 5, 1000, 131072):
+        assert abs(np.linalg.norm(oracle.rope(q, pos)) - np.linalg.norm(q)) < 1e-12
+    # the score depends only on the position difference
+    s1 = oracle.rope(q, 40) @ oracle.rope(k, 13)
+    s2 = oracle.rope(q, 40 + 777) @ oracle.rope(k, 13 + 777)
+    assert abs(s1 - s2) < 1e-11
+    # and it does depend on it (catches a rotation that ignores positions)
+    assert abs(s1 - oracle.rope(q, 41) @ oracle.rope(k, 13)) > 1e-6
+    np.testing.assert_array_equal(oracle.rope(q, 0), q)
+
+
+# ---------------------------------------------------------------------------
+# softmax / attention invariants
+# ---------------------------------------------------------------------------
+
+def test_absorbed_form_equals_unabsorbed():
+    """Matrix absorption (yololab.net section '矩陣吸收') is associativity."""
+    rng = np.random.default_rng(5)
+    inp, ps = _rand_case(rng, B=1, H=3, d_h=6, d_c=12, d_v=5, d_r=4, n_branch=3, lens=(9,),
+                         branch_scale=0.6)
+    got = oracle.decode(inp, page_size=ps)
+    L = 9
+    rows = np.argsort(inp["tok_pos"])
+    C, K = inp["c_kv"][rows], inp["k_rope"][rows]
+    kr = oracle.rope(K, np.arange(L))
+    scale = 1 / math.sqrt(6 + 4)
+    for h in range(3):
+        q_lat = inp["q_nope"][0, h] @ inp["W_UK"][h]                    # [d_c]
+        qr = oracle.rope(inp["q_rope"][0, h], inp["q_pos"][0])
+        o_lat = np.zeros(12)
+        for br in range(3):
+            cols = slice(4 * br, 4 * br + 4)
+            s = scale * (C[:, cols] @ q_lat[cols] + kr @ qr)
+            p = np.exp(s - s.max())
+            o_lat[cols] = 0.6 * (p / p.sum()) @ C[:, cols]
+        out = o_lat @ inp["W_UV"][h]
+        np.testing.assert_allclose(got[(0, h)], out, rtol=1e-10, atol=1e-12)
+
+
+def test_softmax_weights_sum_to_one():
+    """Equal cached rows: every token has the same value, so out = V(c) iff weights sum to 1."""
+    rng = np.random.default_rng(6)
+    inp, ps = _rand_case(rng, B=1, H=2, lens=(7,))
+    c = rng.standard_normal(8)
+    inp["c_kv"][:] = c
+    got = oracle.decode(inp, page_size=ps)
+    for h in range(2):
+        np.testing.assert_allclose(got[(0, h)], c @ inp["W_UV"][h], rtol=1e-12, atol=1e-13)
+
+
+def test_planted_dominant_key():
+    rng = np.random.default_rng(8)
+    inp, ps = _rand_case(rng, B=1, H=1, d_h=4, d_c=8, lens=(6,))
+    inp["q_rope"][:] = 0.0
+    # token 3 gets a logit 40 above the others: q_nope . K_3 * scale = 40 + others ~ 0
+    inp["c_kv"][:] = 0.0
+    qn = inp["q_nope"][0, 0]
+    Wk = inp["W_UK"][0]
+    target = np.linalg.lstsq(Wk, qn / (qn @ qn), rcond=None)[0]  # c with K = W_UK c ~ q direction
+    row3 = int(np.where(inp["tok_pos"] == 3)[0][0])
+    scale = 1 / math.sqrt(4 + 4)
+    K3 = Wk @ target
+    inp["c_kv"][row3] = target * (40.0 / (scale * (qn @ K3)))
+    got = oracle.decode(inp, page_size=ps)[(0, 0)]
+    v3 = inp["c_kv"][row3] @ inp["W_UV"][0]
+    np.testing.assert_allclose(got, v3, rtol=1e-15 + 1e-16, atol=6 * math.exp(-40) * np.abs(v3).max() + 1e-15)
+
+
+def test_mlra_identical_branches_equal_mla():
+    """Four identical branches with weight 1/4 reduce to MLA on one block (wispaper.ai section 2.1)."""
+    rng = np.random.default_rng(9)
+    inp1, ps = _rand_case(rng, B=1, H=2, d_h=4, d_c=4, d_v=3, lens=(5,))
+    inp4 = dict(inp1)
+    inp4["c_kv"] = np.tile(inp1["c_kv"], (1, 4))
+    inp4["W_UK"] = np.tile(inp1["W_UK"], (1, 1, 4))
+    inp4["W_UV"] = np.tile(inp1["W_UV"], (1, 4, 1))
+    inp4["n_branch"], inp4["branch_scale"] = 4, 0.25
+    a = oracle.decode(inp1, page_size=ps)
+    b = oracle.decode(inp4, page_size=ps)
+    assert _max_err(a, b) <= 1e-12
+
+
+def test_mlra_one_branch_is_mla_and_branches_matter():
+    rng = np.random.default_rng(10)
+    inp, ps = _rand_case(rng, n_branch=1)
+    a = oracle.decode(inp, page_size=ps)
+    b = oracle.decode(dict(inp, n_branch=2, branch_scale=1.0), page_size=ps)
+    assert _max_err(a, b) > 1e-3      # separate softmaxes are a different function
+
+
+def test_page_table_permutation_invariance():
+    rng = np.random.default_rng(11)
+    inp, ps = _rand_case(rng, lens=(9, 4))
+    a = oracle.decode(inp, page_size=ps)
+    perm = rng.permutation(inp["num_pages"])
+    pt = inp["page_table"].copy()
+    pt[pt >= 0] = perm[pt[pt >= 0]]
+    b = oracle.decode(dict(inp, page_table=pt), page_size=ps)
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_gather_rejects_unwritten_slot():
+    rng = np.random.default_rng(12)
+    inp, ps = _rand_case(rng, lens=(4, 4))
+    with pytest.raises(ValueError):
+        oracle.decode(dict(inp, seq_lens=np.array([5, 4])), page_size=ps)
+
+
+# ---------------------------------------------------------------------------
+# token compression
+# ---------------------------------------------------------------------------
+
+def test_latent_append_brute_force():
+    rng = np.random.default_rng(13)
+    B, D, d_c, d_r = 2, 5, 4, 4
+    h = rng.standard_normal((B, D))
+    Wd = rng.standard_normal((D, d_c))
+    Wr = rng.standard_normal((D, d_r))
+    pos = np.array([3, 250])
+    c, k_rot, k_raw = oracle.latent_append(h, Wd, Wr, pos)
+    for b in range(B):
+        cb = [sum(h[b, k] * Wd[k, j] for k in range(D)) for j in range(d_c)]
+        kb = [sum(h[b, k] * Wr[k, j] for k in range(D)) for j in range(d_r)]
+        np.testing.assert_allclose(c[b], cb, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(k_raw[b], kb, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(k_rot[b], brute_rope(kb, pos[b], 10000.0), rtol=0, atol=1e-12)
+
+
+def test_bytes_per_cached_token():
+    """576 stored dims (512 latent + 64 rope) in bf16 = 1152 B per token."""
+    from mlra_latent_kv_b200 import synth
+    w = synth.workload("dsv2_contiguous")
+    assert synth.cache_bytes_per_token(w) == 1152
+    # MHA with 32 heads of 128 keeps 2*4096 values per token; the latent keeps 576
+    assert 2 * 32 * 128 / (w.d_c + w.d_r) > 14
+
+
+# ---------------------------------------------------------------------------
+# plant mistakes in the oracle (on the CPU) and check the pins catch them
+# ---------------------------------------------------------------------------
+
+def _pins_pass():
+    try:
+        test_brute_force_tiny(2, 0.7)
+        for c in _golden()["cases"]:
+            test_golden_worked_example(c)
+        for c in _golden()["rope_cases"]:
+            test_golden_rope(c)
+        test_rope_matches_complex_multiplication()
+        test_mlra_identical_branches_equal_mla()
+        test_softmax_weights_sum_to_one()
+    except AssertionError:
+        return False
+    return True
+
+
+def test_planted_mistakes(monkeypatch):
+    assert _pins_pass()
+    orig_rope = mla_oracle.rope
+
+    def rope_wrong_sign(x, pos, base=10000.0):
+        return orig_rope(x, -np.asarray(pos, dtype=np.float64), base)
+
+    def rope_half_index(x, pos, base=10000.0):
+        return orig_rope(x, np.asarray(pos, dtype=np.float64) * 2, base)
+
+    orig_attend = mla_oracle.attend_sequence
+
+    def attend_no_rope(q_nope, q_rope, *a, **k):
+        return orig_attend(q_nope, np.zeros_like(np.asarray(q_rope, dtype=np.float64)), *a, **k)
+
+    def attend_transposed_wuv(q_nope, q_rope, q_pos, W_UK, W_UV, C, K, heads, **k):
+        Wv = np.asarray(W_UV, dtype=np.float64)
+        if Wv.shape[1] == Wv.shape[2]:
+            Wv = np.swapaxes(Wv, 1, 2)
+        else:
+            Wv = Wv[:, ::-1, :]
+        return orig_attend(q_nope, q_rope, q_pos, W_UK, Wv, C, K, heads, **k)
+
+    def attend_scale_sqrt_dh(*a, softmax_scale=None, **k):
+        qn = a[0]
+        return orig_attend(*a, softmax_scale=1.0 / math.sqrt(np.asarray(qn).shape[-1]), **k)
+
+    for name, fn in [("rope", rope_wrong_sign), ("rope", rope_half_index),
+                     ("attend_sequence", attend_no_rope),
+                     ("attend_sequence", attend_transposed_wuv),
+                     ("attend_sequence", attend_scale_sqrt_dh)]:
+        with monkeypatch.context() as m:
+            m.setattr(mla_oracle, name, fn)
+            m.setattr(oracle, name, fn)
+            assert not _pins_pass(), f"planted mistake in {name} ({fn.__name__}) went unnoticed"
+    assert _pins_pass()
