@@ -1,0 +1,199 @@
+/*
+ * mlra.h -- C ABI of libmlra: latent-KV (MLA / MLRA-n) single-token decode
+ * attention over a compressed, paged cache, for NVIDIA B200 (sm_100a).
+ *
+ * Method (pages cited by site, title, section):
+ *   - yololab.net, "超越 GQA 的推理革命：DeepSeek 如何用 MLA 重新定義 LLM 的記憶體
+ *     極限？": section "1. 鍵值聯合低秩壓縮" (each token caches only a latent
+ *     c_KV), section "2. 解耦旋轉位置編碼" (a small RoPE'd key k_rope is kept
+ *     beside it, uncompressed), section "矩陣吸收：推理加速的最後一哩路" (W_UK is
+ *     folded into the query and W_UV applied after attention, so per-head K/V
+ *     are never formed).
+ *   - wispaper.ai, "MLRA：突破 MLA 并行瓶颈，长文本解码提速 280%", section
+ *     "2.1 架构拆解": the latent is cut into branches, each with its own
+ *     softmax, and the output is the weighted sum of the branch outputs.
+ *
+ * Conventions for every entry point
+ *   - Pointers named in a comment as [a, b, ...] are DEVICE pointers to dense
+ *     row-major arrays with those extents (last index fastest), 16-byte aligned.
+ *     Element type: the dims' dtype (bf16 or fp32) for floating arrays, int32
+ *     for index arrays.  Nothing is retained after the call returns except the
+ *     host-side cache of TMA descriptors keyed by (pointer, extents).
+ *   - Ownership: the caller allocates and frees every buffer, including the
+ *     workspace.  The library allocates no device memory in any call.
+ *   - Asynchrony: kernels are enqueued on `stream`; the call returns before
+ *     they finish.  Host-side argument errors are detected before anything is
+ *     enqueued and leave every buffer untouched.
+ *   - Errors: every call returns an mlra_status; mlra_last_error() gives the
+ *     message of the last failure on the calling thread.  Errors found on the
+ *     device (a page id outside [0, num_pages), a bounded wait that gave up)
+ *     are recorded in the first 16 bytes of the workspace and read with
+ *     mlra_check_status().  The workspace must be zero-filled once before its
+ *     first use; mlra_check_status() clears what it reports.
+ */
+#ifndef MLRA_H_
+#define MLRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MLRA_API __attribute__((visibility("default")))
+#else
+#define MLRA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLRA_OK = 0,
+  MLRA_ERR_INVALID_ARG = 1,  /* null pointer, bad extent, misaligned pointer */
+  MLRA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement */
+  MLRA_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace_bytes() figure */
+  MLRA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  MLRA_ERR_DEVICE_CHECK = 5, /* a device-side range check fired (see mlra_check_status) */
+  MLRA_ERR_TIMEOUT = 6       /* a device-side bounded wait gave up */
+} mlra_status;
+
+typedef enum { MLRA_F32 = 0, MLRA_BF16 = 1 } mlra_dtype;
+
+/* Which attention kernel family runs.  AUTO picks the tcgen05 kernels when the
+ * shape is one they implement (bf16, d_c = 512, d_r = 64, H <= 128,
+ * n_branch in {1, 2, 4}) and the CUDA-core kernels otherwise. */
+typedef enum { MLRA_KERNEL_AUTO = 0, MLRA_KERNEL_SIMT = 1, MLRA_KERNEL_TC = 2 } mlra_kernel;
+
+/* Shape and parameters of a decode batch.
+ *   B            sequences in the batch
+ *   H            query heads
+ *   d_h          per-head query/key content width (q_nope, rows of W_UK)
+ *   d_v          per-head value width (columns of W_UV)
+ *   d_c          latent width c_KV (all branches together)
+ *   d_r          decoupled RoPE key width (even)
+ *   n_branch     MLRA branches; 1 = MLA.  Branch br owns latent columns
+ *                [br*d_c/n_branch, (br+1)*d_c/n_branch)
+ *   page_size    tokens per cache page (64)
+ *   max_pages_per_seq  row length of page_table
+ *   num_pages    pages in the cache pool
+ *   softmax_scale  logit scale; 0 selects 1/sqrt(d_h + d_r)
+ *   branch_scale   weight of each branch output in the sum (1 for MLA)
+ *   rope_base      RoPE base; 0 selects 10000
+ *   dtype        element type of caches, queries, weights and outputs
+ *   num_splits   split-KV workers; 0 = chosen from the device's SM count
+ *   kernel       an mlra_kernel value                                      */
+typedef struct {
+  int B, H, d_h, d_v, d_c, d_r;
+  int n_branch;
+  int page_size;
+  int max_pages_per_seq;
+  int num_pages;
+  float softmax_scale;
+  float branch_scale;
+  float rope_base;
+  int dtype;
+  int num_splits;
+  int kernel;
+} mlra_dims;
+
+/* Bytes of workspace a decode call with these dims needs (0 on invalid dims;
+ * the reason is in mlra_last_error()).  With num_splits = 0 it queries the
+ * current device. */
+MLRA_API size_t mlra_workspace_bytes(const mlra_dims* dims);
+
+/* mla_decode -- one decode step of MLA (n_branch must be 1; branch_scale is
+ * taken as 1).  Absorbed form, yololab.net section "矩陣吸收":
+ *   q_lat[b,h]  = q_nope[b,h] . W_UK[h]                         (d_c)
+ *   q_rot[b,h]  = RoPE(q_rope[b,h], q_pos[b])                   (d_r)
+ *   s[b,h,t]    = scale * (q_lat . c[b,t] + q_rot . k[b,t]),  t < seq_lens[b]
+ *   o_lat[b,h]  = softmax_t(s) . c[b,:]                         (d_c)
+ *   out[b,h]    = o_lat[b,h] . W_UV[h]                          (d_v)
+ * where c[b,t] = latent_cache[page_table[b][t/64]][t%64] and k[b,t] the same
+ * slot of rope_cache (stored rotated at position t).  seq_lens[b] = 0 gives a
+ * zero row.
+ *   q_nope [B,H,d_h]   q_rope [B,H,d_r] (un-rotated)   q_pos [B] int32
+ *   W_UK [H,d_h,d_c]   W_UV [H,d_c,d_v]
+ *   latent_cache [num_pages,page_size,d_c]   rope_cache [num_pages,page_size,d_r]
+ *   page_table [B,max_pages_per_seq] int32   seq_lens [B] int32
+ *   out [B,H,d_v]  (written)
+ *   workspace: >= mlra_workspace_bytes(dims) bytes, 256-byte aligned. */
+MLRA_API mlra_status mla_decode(const mlra_dims* dims, const void* q_nope, const void* q_rope,
+                       const int32_t* q_pos, const void* W_UK, const void* W_UV,
+                       const void* latent_cache, const void* rope_cache,
+                       const int32_t* page_table, const int32_t* seq_lens, void* out,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* mlra_decode -- MLRA-n decode (wispaper.ai section "2.1 架构拆解"): the same
+ * arguments as mla_decode; each branch br runs its own softmax over
+ *   s_br = scale * (q_lat[br cols] . c[br cols] + q_rot . k)
+ * (the rope score is shared by all branches) and
+ *   out = sum_br branch_scale * softmax(s_br) . c[br cols] . W_UV[h][br rows]. */
+MLRA_API mlra_status mlra_decode(const mlra_dims* dims, const void* q_nope, const void* q_rope,
+                        const int32_t* q_pos, const void* W_UK, const void* W_UV,
+                        const void* latent_cache, const void* rope_cache,
+                        const int32_t* page_table, const int32_t* seq_lens, void* out,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* mlra_decode_profiled -- mlra_decode that also records stage_events[0..4]
+ * (created by the caller) on `stream`: before query absorption, after it,
+ * after split-KV attention, after the split combine, after the output
+ * up-projection.  stage_events may be NULL. */
+MLRA_API mlra_status mlra_decode_profiled(const mlra_dims* dims, const void* q_nope, const void* q_rope,
+                                 const int32_t* q_pos, const void* W_UK, const void* W_UV,
+                                 const void* latent_cache, const void* rope_cache,
+                                 const int32_t* page_table, const int32_t* seq_lens, void* out,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                                 cudaEvent_t* stage_events);
+
+/* Bytes of workspace latent_append needs for hidden width d_model. */
+MLRA_API size_t latent_append_workspace_bytes(const mlra_dims* dims, int d_model);
+
+/* latent_append -- compress one new token per sequence into the cache
+ * (yololab.net sections "1. 鍵值聯合低秩壓縮" and "2. 解耦旋轉位置編碼"):
+ *   x = h[b] . [W_DKV | W_KR]           (fp32 accumulate)
+ *   latent_cache[slot] = x[:d_c]          rope_cache[slot] = RoPE(x[d_c:], pos[b])
+ * with slot = (page_table[b][pos[b]/page_size], pos[b] % page_size), both
+ * rounded to the dtype (round to nearest even).  seq_lens is not touched; a
+ * caller that then attends the new token passes seq_lens[b] = pos[b] + 1.
+ *   h [B,d_model]   W_DKV [d_model,d_c]   W_KR [d_model,d_r]   pos [B] int32
+ *   page_table [B,max_pages_per_seq] int32; the caches are written at one slot
+ *   per sequence and nowhere else. */
+MLRA_API mlra_status latent_append(const mlra_dims* dims, int d_model, const void* h, const void* W_DKV,
+                          const void* W_KR, const int32_t* pos, const int32_t* page_table,
+                          void* latent_cache, void* rope_cache, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream);
+
+/* latent_store -- write already-compressed tokens into the paged cache
+ * (prefill, or restoring a cache): for i < n_tokens, token row i goes to
+ * sequence tok_seq[i] at position tok_pos[i]:
+ *   latent_cache[slot] = c_kv[i]   (copied bit for bit)
+ *   rope_cache[slot]   = RoPE(k_rope[i], tok_pos[i])   (rounded to nearest even)
+ *   c_kv [n_tokens,d_c]   k_rope [n_tokens,d_r] (un-rotated)
+ *   tok_seq, tok_pos [n_tokens] int32
+ * workspace: at least 256 bytes (device error record). */
+MLRA_API mlra_status latent_store(const mlra_dims* dims, int n_tokens, const void* c_kv, const void* k_rope,
+                         const int32_t* tok_seq, const int32_t* tok_pos, const int32_t* page_table,
+                         void* latent_cache, void* rope_cache, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, reads the device error record in `workspace`, clears
+ * it and returns MLRA_OK, MLRA_ERR_DEVICE_CHECK or MLRA_ERR_TIMEOUT (the
+ * message, with the first offending index, goes to mlra_last_error()). */
+MLRA_API mlra_status mlra_check_status(void* workspace, cudaStream_t stream);
+
+/* Message of the last error on the calling thread ("" if none). */
+MLRA_API const char* mlra_last_error(void);
+
+/* Frees host-side caches (TMA descriptors).  Safe to call at any time when no
+ * call is in progress on another thread. */
+MLRA_API void mlra_shutdown(void);
+
+/* ABI version: 1. */
+MLRA_API int mlra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLRA_H_ */

@@ -1,0 +1,172 @@
+"""ctypes binding of libmlra (include/mlra.h): argument marshalling only.
+
+Every computation runs in the CUDA library; this module turns torch tensors
+into device pointers and status codes into exceptions.  It fails loudly if the
+library is missing -- there is no other implementation behind these names.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmlra.so")
+
+MLRA_OK = 0
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
+                5: "DEVICE_CHECK", 6: "TIMEOUT"}
+DTYPES = {"f32": 0, "bf16": 1}
+KERNELS = {"auto": 0, "simt": 1, "tc": 2}
+
+
+class MlraError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libmlra {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d_h", ctypes.c_int), ("d_v", ctypes.c_int),
+                ("d_c", ctypes.c_int), ("d_r", ctypes.c_int), ("n_branch", ctypes.c_int),
+                ("page_size", ctypes.c_int), ("max_pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float), ("branch_scale", ctypes.c_float),
+                ("rope_base", ctypes.c_float), ("dtype", ctypes.c_int), ("num_splits", ctypes.c_int),
+                ("kernel", ctypes.c_int)]
+
+
+def make_dims(*, B, H, d_h, d_v, d_c, d_r, max_pages_per_seq, num_pages, n_branch=1, page_size=64,
+              softmax_scale=0.0, branch_scale=1.0, rope_base=0.0, dtype="bf16", num_splits=0,
+              kernel="auto") -> Dims:
+    return Dims(B, H, d_h, d_v, d_c, d_r, n_branch, page_size, max_pages_per_seq, num_pages,
+                float(softmax_scale), float(branch_scale), float(rope_base), DTYPES[dtype], num_splits,
+                KERNELS[kernel])
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+_DIMS = ctypes.POINTER(Dims)
+_DECODE_ARGS = [_DIMS, _P, _P, _I32P, _P, _P, _P, _P, _I32P, _I32P, _P, _P, _SZ, _P]
+
+SIGNATURES = {
+    "mlra_workspace_bytes": (_SZ, [_DIMS]),
+    "mla_decode": (ctypes.c_int, _DECODE_ARGS),
+    "mlra_decode": (ctypes.c_int, _DECODE_ARGS),
+    "mlra_decode_profiled": (ctypes.c_int, _DECODE_ARGS + [_P]),
+    "latent_append_workspace_bytes": (_SZ, [_DIMS, ctypes.c_int]),
+    "latent_append": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
+    "latent_store": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _I32P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
+    "mlra_check_status": (ctypes.c_int, [_P, _P]),
+    "mlra_last_error": (ctypes.c_char_p, []),
+    "mlra_shutdown": (None, []),
+    "mlra_version": (ctypes.c_int, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if libmlra.so has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m mlra_latent_kv_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().mlra_last_error().decode()
+
+
+def _check(status: int):
+    if status != MLRA_OK:
+        raise MlraError(status, last_error())
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def workspace_bytes(dims: Dims) -> int:
+    n = lib().mlra_workspace_bytes(ctypes.byref(dims))
+    if n == 0:
+        raise MlraError(1, last_error())
+    return int(n)
+
+
+def _decode(fn, dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table, seq_lens, out,
+            workspace, workspace_nbytes=None, stream=None, extra=()):
+    nbytes = workspace_nbytes if workspace_nbytes is not None else \
+        workspace.numel() * workspace.element_size()
+    _check(fn(ctypes.byref(dims), _ptr(q_nope), _ptr(q_rope), _ptr(q_pos), _ptr(W_UK), _ptr(W_UV),
+              _ptr(latent_cache), _ptr(rope_cache), _ptr(page_table), _ptr(seq_lens), _ptr(out),
+              _ptr(workspace), nbytes, _stream(stream), *extra))
+
+
+def mla_decode(dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table, seq_lens, out,
+               workspace, workspace_nbytes=None, stream=None):
+    _decode(lib().mla_decode, dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table,
+            seq_lens, out, workspace, workspace_nbytes, stream)
+
+
+def mlra_decode(dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table, seq_lens, out,
+                workspace, workspace_nbytes=None, stream=None):
+    _decode(lib().mlra_decode, dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table,
+            seq_lens, out, workspace, workspace_nbytes, stream)
+
+
+def mlra_decode_profiled(dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table, seq_lens,
+                         out, workspace, events, workspace_nbytes=None, stream=None):
+    """``events``: five torch.cuda.Event(enable_timing=True), already recorded once (so they exist)."""
+    arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+    _decode(lib().mlra_decode_profiled, dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache,
+            page_table, seq_lens, out, workspace, workspace_nbytes, stream, extra=(ctypes.cast(arr, _P),))
+
+
+def append_workspace_bytes(dims: Dims, d_model: int) -> int:
+    n = lib().latent_append_workspace_bytes(ctypes.byref(dims), d_model)
+    if n == 0:
+        raise MlraError(1, last_error())
+    return int(n)
+
+
+def latent_append(dims, d_model, h, W_DKV, W_KR, pos, page_table, latent_cache, rope_cache, workspace,
+                  workspace_nbytes=None, stream=None):
+    nbytes = workspace_nbytes if workspace_nbytes is not None else workspace.numel() * workspace.element_size()
+    _check(lib().latent_append(ctypes.byref(dims), int(d_model), _ptr(h), _ptr(W_DKV), _ptr(W_KR), _ptr(pos),
+                               _ptr(page_table), _ptr(latent_cache), _ptr(rope_cache), _ptr(workspace), nbytes,
+                               _stream(stream)))
+
+
+def latent_store(dims, n_tokens, c_kv, k_rope, tok_seq, tok_pos, page_table, latent_cache, rope_cache, workspace,
+                 workspace_nbytes=None, stream=None):
+    nbytes = workspace_nbytes if workspace_nbytes is not None else workspace.numel() * workspace.element_size()
+    _check(lib().latent_store(ctypes.byref(dims), int(n_tokens), _ptr(c_kv), _ptr(k_rope), _ptr(tok_seq),
+                              _ptr(tok_pos), _ptr(page_table), _ptr(latent_cache), _ptr(rope_cache),
+                              _ptr(workspace), nbytes, _stream(stream)))
+
+
+def check_status(workspace, stream=None) -> None:
+    _check(lib().mlra_check_status(_ptr(workspace), _stream(stream)))
+
+
+def version() -> int:
+    return int(lib().mlra_version())

@@ -1,0 +1,25 @@
+// tcgen05 (5th-generation tensor core) split-KV latent attention for sm_100a.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "launch.h"
+
+namespace mlra {
+
+// Query rows per sequence the tcgen05 kernels read (heads padded with zero rows).
+constexpr int kTcHeads = 128;
+
+// Whether the tcgen05 attention kernels implement this shape.
+bool tc_supported(int dtype, int H, int d_c, int d_r, int n_branch, int d_h, int d_v);
+
+// Launch the tcgen05 split-KV attention: same partial-result contract as the
+// CUDA-core kernel (slot c + b per worker piece, m/l per branch in log2 units).
+cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop, const int* page_table,
+                             const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
+                             cudaStream_t st);
+
+// Frees the host-side tensor-map cache.
+void tc_shutdown();
+
+}  // namespace mlra

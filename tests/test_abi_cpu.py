@@ -1,0 +1,121 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/mlra.h declares, and rejects bad arguments before
+enqueueing anything (fake device pointers are never dereferenced on these
+paths)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from mlra_latent_kv_b200 import abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return abi.lib()
+
+
+def declared_symbols():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names += re.findall(r"MLRA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), f"libmlra.so does not export {n}"
+        assert n in abi.SIGNATURES, f"binding has no signature for {n}"
+    assert abi.version() == 1
+
+
+def _dims(**kw):
+    base = dict(B=4, H=128, d_h=128, d_v=128, d_c=512, d_r=64, max_pages_per_seq=8, num_pages=32,
+                num_splits=74, dtype="bf16")
+    base.update(kw)
+    return abi.make_dims(**base)
+
+
+FAKE = 1 << 20  # 256-byte aligned, never dereferenced on validation paths
+
+
+def _decode(fn, dims, ws_bytes, **over):
+    args = dict(q_nope=FAKE, q_rope=FAKE, q_pos=FAKE, W_UK=FAKE, W_UV=FAKE, latent_cache=FAKE, rope_cache=FAKE,
+                page_table=FAKE, seq_lens=FAKE, out=FAKE, workspace=FAKE)
+    args.update(over)
+    return fn(ctypes.byref(dims), args["q_nope"], args["q_rope"], args["q_pos"], args["W_UK"], args["W_UV"],
+              args["latent_cache"], args["rope_cache"], args["page_table"], args["seq_lens"], args["out"],
+              args["workspace"], ws_bytes, None)
+
+
+def test_workspace_layout_formula(L):
+    # simt path, fp32: err 256 | q B*H*(d_c+d_r)*4 | o_part slots*H*d_c*4 | ml slots*nbr*2*H*4 | o_lat B*H*d_c*4
+    d = _dims(dtype="f32", kernel="simt", num_splits=10, B=3, H=8, d_h=32, d_v=32, d_c=64, d_r=16)
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    slots = 10 + 3 - 1
+    exp = 256
+    exp = r(exp + 3 * 8 * 80 * 4)
+    exp = r(exp + slots * 8 * 64 * 4)
+    exp = r(exp + slots * 1 * 2 * 8 * 4)
+    exp = r(exp + 3 * 8 * 64 * 4)
+    assert abi.workspace_bytes(d) == exp
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(d_r=3), 1), (dict(B=0), 1), (dict(n_branch=3), 1), (dict(dtype="bf16", page_size=32), 2),
+    (dict(d_c=520), 2), (dict(d_r=128), 2), (dict(softmax_scale=-1.0), 1), (dict(num_pages=0), 1),
+])
+def test_bad_dims_rejected(L, over, status):
+    page_size = over.pop("page_size", 64)
+    d = _dims(**over)
+    d.page_size = page_size
+    st = _decode(L.mlra_decode, d, 1 << 40)
+    assert st == status, abi.last_error()
+    assert abi.last_error()
+
+
+def test_null_and_misaligned_pointers(L):
+    d = _dims()
+    assert _decode(L.mlra_decode, d, 1 << 40, q_nope=None) == 1
+    assert "q_nope" in abi.last_error()
+    assert _decode(L.mlra_decode, d, 1 << 40, out=FAKE + 8) == 1
+    assert "aligned" in abi.last_error()
+    assert _decode(L.mlra_decode, d, 1 << 40, workspace=FAKE + 16) == 1
+
+
+def test_small_workspace_rejected(L):
+    d = _dims()
+    need = abi.workspace_bytes(d)
+    assert _decode(L.mlra_decode, d, need - 1) == 3
+    assert str(need) in abi.last_error()
+
+
+def test_mla_decode_needs_one_branch(L):
+    d = _dims(n_branch=4, branch_scale=0.5)
+    assert _decode(L.mla_decode, d, 1 << 40) == 1
+
+
+def test_tc_request_outside_tc_shapes_is_unsupported(L):
+    d = _dims(dtype="f32", kernel="tc")
+    assert _decode(L.mlra_decode, d, 1 << 40) == 2
+
+
+def test_append_and_store_validation(L):
+    d = _dims()
+    assert L.latent_append_workspace_bytes(ctypes.byref(d), 0) == 0
+    n = L.latent_append_workspace_bytes(ctypes.byref(d), 5120)
+    assert n == 256 + (80 * 4 * 576 * 4 + 255) // 256 * 256
+    st = L.latent_append(ctypes.byref(d), 5120, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n - 1, None)
+    assert st == 3
+    st = L.latent_store(ctypes.byref(d), -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None)
+    assert st == 1
+    st = L.latent_store(ctypes.byref(d), 10, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None)
+    assert st == 1

@@ -1,0 +1,150 @@
+"""GPU parity of the decode path against the fp64 oracle, through the C ABI.
+
+Reduced sizes span several 64-token pages with ragged tails and compare every
+(b, h); the full workload sizes compare sampled (b, h) rows in the launch
+configuration the benchmark times.  Tolerance (bf16 cache, fp32 accumulate):
+max|gpu - oracle| <= 1e-2 * max|oracle| + 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mlra_latent_kv_b200 import abi, synth
+from mlra_latent_kv_b200.session import DecodeSession
+
+from _support import compare, oracle_inputs, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = ["simt", "auto"]
+
+
+def run_case(w, kernel="auto", num_splits=0, pairs=None, inp=None):
+    inp = inp if inp is not None else synth.make_inputs(w)
+    s = DecodeSession(w, inp, kernel=kernel, num_splits=num_splits)
+    out = s.step().clone()
+    torch.cuda.synchronize()
+    s.check()
+    ref = oracle.decode(oracle_inputs(w, inp), pairs)
+    err, tol = compare(out, ref)
+    return err, tol, out, ref, s
+
+
+REDUCED = {
+    "tiny_mla_fp32": dict(),
+    "dsv2_contiguous": dict(B=3, seq_len=300),
+    "paged_varlen_h32": dict(B=6, seq_len_range=(1, 700)),
+    "mlra4": dict(B=2, seq_len=333),
+    "longctx_append": dict(B=2, seq_len=200),
+}
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("name", list(REDUCED))
+def test_reduced_workloads(name, kernel):
+    w = synth.workload(name).with_(**REDUCED[name])
+    err, tol, out, ref, _ = run_case(w, kernel)
+    assert err <= tol, f"{name}/{kernel}: max err {err:.3e} > tol {tol:.3e} (rel l2 {rel_l2(out, ref):.2e})"
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("H", [128, 64, 32, 8])
+def test_edge_lengths_mla(H, kernel):
+    lens = [0, 1, 63, 64, 65, 127, 128, 129]
+    w = synth.workload("dsv2_contiguous").with_(B=len(lens), H=H, seq_len_range=(1, 2), paged=True, nan_tails=True)
+    inp = synth.make_inputs(w.with_(seq_len_range=None, seq_len=max(lens)))
+    # rebuild with explicit lengths: draw at max length, keep the first L_b tokens of each sequence
+    keep = np.concatenate([np.arange(max(lens)) < L for L in lens])
+    for k in ("c_kv", "k_rope", "tok_seq", "tok_pos"):
+        inp[k] = inp[k][torch.from_numpy(keep)]
+    inp["seq_lens"] = torch.tensor(lens, dtype=torch.int32)
+    inp["attn_lens"] = inp["seq_lens"].clone()
+    inp["q_pos"] = inp["seq_lens"].clone()
+    err, tol, out, ref, _ = run_case(w, kernel, inp=inp)
+    assert err <= tol, f"H={H}/{kernel}: {err:.3e} > {tol:.3e}"
+    assert torch.all(out[0] == 0), "empty sequence must give a zero row"
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("nbr,bscale", [(2, 0.7), (4, 0.5)])
+def test_mlra_branches(nbr, bscale, kernel):
+    w = synth.workload("mlra4").with_(B=3, seq_len_range=(60, 260), n_branch=nbr, branch_scale=bscale)
+    err, tol, out, ref, _ = run_case(w, kernel)
+    assert err <= tol
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("G", [1, 3, 7, 200])
+def test_split_counts(G, kernel):
+    """Worker counts below, near and far above the page count exercise the split plan."""
+    w = synth.workload("paged_varlen_h32").with_(B=5, seq_len_range=(1, 400))
+    err, tol, *_ = run_case(w, kernel, num_splits=G)
+    assert err <= tol
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_page_permutation_bitwise(kernel):
+    """Moving pages around the pool (page table permuted with them) changes no output bit."""
+    w = synth.workload("dsv2_contiguous").with_(B=3, seq_len=250, paged=True)
+    inp = synth.make_inputs(w)
+    s1 = DecodeSession(w, inp, kernel=kernel)
+    o1 = s1.step().clone()
+    perm = torch.randperm(inp["num_pages"], generator=torch.Generator().manual_seed(5)).to(torch.int32)
+    pt = inp["page_table"].clone()
+    m = pt >= 0
+    pt[m] = perm[pt[m].long()]
+    s2 = DecodeSession(w, dict(inp, page_table=pt), kernel=kernel)
+    o2 = s2.step().clone()
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_dominant_key_is_selected(kernel):
+    """A planted key 120 logits above the rest (exp(120) overflows fp32): the
+    output is that token's value row, so the running-max subtraction works."""
+    w = synth.workload("dsv2_contiguous").with_(B=1, H=128, seq_len=200)
+    inp = synth.make_inputs(w)
+    inp["q_rope"].zero_()
+    q_lat = inp["q_nope"][0, 0].double() @ inp["W_UK"][0].double()
+    scale = 1.0 / np.sqrt(w.d_h + w.d_r)
+    c77 = q_lat / (q_lat @ q_lat) * (120.0 / scale)
+    inp["c_kv"][77] = c77.to(inp["c_kv"].dtype)
+    ref = oracle.decode(oracle_inputs(w, inp), [(0, 0)])
+    v77 = inp["c_kv"][77].double().numpy() @ inp["W_UV"][0].double().numpy()
+    np.testing.assert_allclose(ref[(0, 0)], v77, rtol=1e-6, atol=1e-6)
+    s = DecodeSession(w, inp, kernel=kernel)
+    out = s.step()
+    err, tol = compare(out, ref)
+    assert err <= tol
+
+
+def test_device_check_bad_page_id():
+    w = synth.workload("dsv2_contiguous").with_(B=2, seq_len=100)
+    inp = synth.make_inputs(w)
+    s = DecodeSession(w, inp, kernel="simt")
+    s.page_table[1, 1] = 10_000_000  # outside the pool
+    s.decode()
+    with pytest.raises(abi.MlraError) as ei:
+        s.check()
+    assert ei.value.status == 5
+    s.check()  # cleared
+
+
+FULL_PAIRS = {
+    "tiny_mla_fp32": None,
+    "dsv2_contiguous": [(0, 0), (5, 77), (31, 127), (17, 3)],
+    "paged_varlen_h32": [(0, 0), (13, 31), (40, 7), (63, 16)],
+    "mlra4": [(0, 0), (11, 64), (31, 127)],
+    "longctx_append": [(0, 0), (3, 127), (1, 50)],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL_PAIRS))
+def test_full_size_sampled(name):
+    """Full workload sizes, default launch configuration (the one the benchmark times)."""
+    w = synth.workload(name)
+    err, tol, out, ref, _ = run_case(w, "auto", pairs=FULL_PAIRS[name])
+    assert err <= tol, f"{name}: {err:.3e} > {tol:.3e}"
+    assert torch.isfinite(out.float()).all()
