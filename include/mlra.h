@@ -177,6 +177,34 @@ MLRA_API mlra_status latent_store(const mlra_dims* dims, int n_tokens, const voi
                          void* latent_cache, void* rope_cache, void* workspace,
                          size_t workspace_bytes, cudaStream_t stream);
 
+/* latent_append_noalloc -- latent_append for callers that cannot allocate
+ * device memory: a serving engine that reserved all HBM for its cache pool up
+ * front and forbids later cudaMalloc (late allocations fragment memory or
+ * fail once the pool is full), a decode loop that must not hit the device-wide
+ * synchronisation cudaMalloc/cudaFree can cause, or a plugin host that hands
+ * over input and output buffers but no allocator.  It computes exactly what
+ * latent_append computes (same kernels, same result bits) but takes no
+ * workspace: its split-K scratch is a fixed device array inside libmlra of
+ * MLRA_NOALLOC_SCRATCH_BYTES (4 MiB), which every GPU that loads the library
+ * holds until the process exits.  There is no counterpart on the pages; this
+ * is an interface convenience only.
+ *   - Scratch needed: ceil(d_model/64) * B * (d_c + d_r) * 4 bytes; a call
+ *     that needs more returns MLRA_ERR_UNSUPPORTED and enqueues nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array.  Each call overwrites the part it uses
+ *     before reading it, so nothing has to start zeroed, but calls whose
+ *     kernels overlap on the GPU (e.g. on two streams) race on it.
+ *   - Device-side range checks still keep every access inside the cache, but
+ *     their reports are not recorded (there is no workspace to hold them).
+ * It allocates nothing and frees nothing. */
+#define MLRA_NOALLOC_SCRATCH_BYTES (4u << 20)
+MLRA_API mlra_status latent_append_noalloc(const mlra_dims* dims, int d_model, const void* h,
+                                           const void* W_DKV, const void* W_KR, const int32_t* pos,
+                                           const int32_t* page_table, void* latent_cache,
+                                           void* rope_cache, cudaStream_t stream);
+
 /* Synchronises `stream`, reads the device error record in `workspace`, clears
  * it and returns MLRA_OK, MLRA_ERR_DEVICE_CHECK or MLRA_ERR_TIMEOUT (the
  * message, with the first offending index, goes to mlra_last_error()). */

@@ -57,6 +57,7 @@ SIGNATURES = {
     "latent_append_workspace_bytes": (_SZ, [_DIMS, ctypes.c_int]),
     "latent_append": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "latent_store": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _I32P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
+    "latent_append_noalloc": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P]),
     "mlra_check_status": (ctypes.c_int, [_P, _P]),
     "mlra_last_error": (ctypes.c_char_p, []),
     "mlra_shutdown": (None, []),
@@ -162,6 +163,15 @@ def latent_store(dims, n_tokens, c_kv, k_rope, tok_seq, tok_pos, page_table, lat
     _check(lib().latent_store(ctypes.byref(dims), int(n_tokens), _ptr(c_kv), _ptr(k_rope), _ptr(tok_seq),
                               _ptr(tok_pos), _ptr(page_table), _ptr(latent_cache), _ptr(rope_cache),
                               _ptr(workspace), nbytes, _stream(stream)))
+
+
+def latent_append_noalloc(dims, d_model, h, W_DKV, W_KR, pos, page_table, latent_cache, rope_cache, stream=None):
+    """latent_append without a workspace, for callers that cannot allocate
+    device memory; its scratch is a fixed array inside the library (see
+    include/mlra.h for the size limit and the sharing rules)."""
+    _check(lib().latent_append_noalloc(ctypes.byref(dims), int(d_model), _ptr(h), _ptr(W_DKV), _ptr(W_KR),
+                                       _ptr(pos), _ptr(page_table), _ptr(latent_cache), _ptr(rope_cache),
+                                       _stream(stream)))
 
 
 def check_status(workspace, stream=None) -> None:

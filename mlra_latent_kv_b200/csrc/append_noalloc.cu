@@ -1,0 +1,89 @@
+// latent_append_noalloc: latent_append for callers that cannot allocate
+// device memory (an engine whose cache pool owns all HBM and forbids later
+// cudaMalloc, a decode loop that must not risk the synchronisation an
+// allocation can cause, a plugin host that passes buffers but no allocator).
+// The split-K partial sums that latent_append keeps in the caller's workspace
+// live here in one fixed, file-scope device array instead.  There is no
+// counterpart on the pages.
+#include <cstdio>
+#include <mutex>
+
+#include "launch.h"
+
+using namespace mlra;
+
+namespace {
+
+// The scratch: every GPU that loads the library holds one copy until exit.
+static __device__ __align__(256) unsigned char g_append_scratch[MLRA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_dev[kMaxDevices] = {};  // device address of g_append_scratch, by device ordinal
+
+// Device address of the scratch on the current device.  Host code cannot use
+// the array's name as an address (it is a host-side stand-in), so the first
+// call on each device asks the runtime for it, with that device current, and
+// keeps the answer.
+cudaError_t scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_dev[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_append_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_dev[dev] = p;
+  }
+  *out = g_scratch_dev[dev];
+  return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" MLRA_API mlra_status latent_append_noalloc(const mlra_dims* dims, int d_model, const void* h,
+                                                      const void* W_DKV, const void* W_KR, const int32_t* pos,
+                                                      const int32_t* page_table, void* latent_cache,
+                                                      void* rope_cache, cudaStream_t stream) {
+  char msg[256];
+  mlra_status st = internal_check_dims(dims);
+  if (st != MLRA_OK) return st;
+  if (d_model < 1) return internal_fail(MLRA_ERR_INVALID_ARG, "d_model must be >= 1");
+  const void* ptrs[] = {h, W_DKV, W_KR, latent_cache, rope_cache};
+  const char* names[] = {"h", "W_DKV", "W_KR", "latent_cache", "rope_cache"};
+  for (int i = 0; i < 5; ++i) {
+    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) {
+      snprintf(msg, sizeof(msg), "%s is NULL or not 16-byte aligned", names[i]);
+      return internal_fail(MLRA_ERR_INVALID_ARG, msg);
+    }
+  }
+  if (pos == nullptr || page_table == nullptr) return internal_fail(MLRA_ERR_INVALID_ARG, "pos/page_table is NULL");
+  const int KS = (d_model + 63) / 64;
+  const size_t need = (size_t)KS * dims->B * (dims->d_c + dims->d_r) * sizeof(float);
+  if (need > MLRA_NOALLOC_SCRATCH_BYTES) {
+    snprintf(msg, sizeof(msg),
+             "latent_append_noalloc: B=%d, d_model=%d, d_c+d_r=%d need %zu bytes of scratch; the fixed scratch "
+             "holds %u bytes (call latent_append with a workspace instead)",
+             dims->B, d_model, dims->d_c + dims->d_r, need, (unsigned)MLRA_NOALLOC_SCRATCH_BYTES);
+    return internal_fail(MLRA_ERR_UNSUPPORTED, msg);
+  }
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof(msg), "latent_append_noalloc: looking up the scratch address: %s", cudaGetErrorString(e));
+    return internal_fail(MLRA_ERR_CUDA, msg);
+  }
+  // pass 1 writes every partial sum pass 2 reads, so the scratch needs no clearing
+  AppendArgs a{dims->B, d_model, dims->d_c, dims->d_r, dims->max_pages_per_seq, dims->num_pages, KS};
+  e = launch_append(dims->dtype, h, W_DKV, W_KR, pos, page_table, latent_cache, rope_cache,
+                    static_cast<float*>(scratch), /*err=*/nullptr, a, internal_rope_table(dims), stream);
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof(msg), "latent_append_noalloc launch: %s", cudaGetErrorString(e));
+    return internal_fail(MLRA_ERR_CUDA, msg);
+  }
+  return MLRA_OK;
+}

@@ -53,3 +53,12 @@ cudaError_t launch_store(int dtype, const void* c_kv, const void* k_rope, const 
                          const RopeTable& tab, cudaStream_t st);
 
 }  // namespace mlra
+
+#include "../../include/mlra.h"
+
+namespace mlra {
+// defined in mlra_api.cu
+mlra_status internal_check_dims(const mlra_dims* d);
+mlra_status internal_fail(mlra_status st, const char* msg);
+RopeTable internal_rope_table(const mlra_dims* d);
+}  // namespace mlra

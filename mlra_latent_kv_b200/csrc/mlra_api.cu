@@ -302,3 +302,10 @@ void mlra_shutdown(void) { tc_shutdown(); }
 int mlra_version(void) { return 1; }
 
 }  // extern "C"
+
+// Internal helpers for entry points defined in other translation units.
+namespace mlra {
+mlra_status internal_check_dims(const mlra_dims* d) { return check_dims(d); }
+mlra_status internal_fail(mlra_status st, const char* msg) { return fail(st, "%s", msg); }
+RopeTable internal_rope_table(const mlra_dims* d) { return rope_table(d); }
+}  // namespace mlra
