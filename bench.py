@@ -168,8 +168,8 @@ def pick_pairs(w, n, seed=0):
 
 def cpu_baseline(w, inp, budget_s: float = 15.0) -> dict:
     """The oracle (as it stands) on a bounded sample of (b, h) pairs, scaled to a full step."""
-    t1 = time_oracle_pairs(w, inp, pick_pairs(w, 1))
-    n = max(1, min(w.B * w.H, int(budget_s / max(t1, 1e-6))))
+    t8 = time_oracle_pairs(w, inp, pick_pairs(w, 8, seed=7)) / 8
+    n = max(1, min(w.B * w.H, int(budget_s / max(t8, 1e-6))))
     pairs = pick_pairs(w, n, seed=1)
     t = time_oracle_pairs(w, inp, pairs)
     per_pair = t / n
@@ -245,24 +245,49 @@ def run_ours(args, w):
 
     K, W = args.steps, args.warmup
     starts, ends = mk(K), mk(K)
-    stage = [mk(5) for _ in range(K)]
-    for evs in stage:  # materialise the raw events before handing them to the library
-        for e in evs:
-            e.record(stream)
+    stage = mk(5)
+    for e in stage:  # materialise the raw events before handing them to the library
+        e.record(stream)
     for _ in range(W):
         flush.fill_(1)
         sess.step()
     torch.cuda.synchronize(dev)
     sess.check()
+    # one decode step captured as a CUDA graph (the library records the stage
+    # events as graph nodes), replayed once per timed step
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            sess.step(events=stage)
+        for _ in range(W):
+            flush.fill_(1)
+            graph.replay()
+        torch.cuda.synchronize(dev)
 
+    def one_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            sess.step(events=stage)
+
+    stage_acc = {"absorb": 0.0, "attention": 0.0, "combine": 0.0, "upproj_incl_fused_combine": 0.0}
+    if sess.appends:
+        stage_acc["append"] = 0.0
     mdist.barrier(dev)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(K):
             flush.fill_(i & 0xFF)
             starts[i].record(stream)
-            sess.step(events=stage[i])
+            one_step()
             ends[i].record(stream)
+            ends[i].synchronize()
+            for name, a, b in (("absorb", 0, 1), ("attention", 1, 2), ("combine", 2, 3),
+                               ("upproj_incl_fused_combine", 3, 4)):
+                stage_acc[name] += stage[a].elapsed_time(stage[b])
+            if sess.appends:
+                stage_acc["append"] += starts[i].elapsed_time(stage[0])
         torch.cuda.synchronize(dev)
     mdist.barrier(dev)
     torch.cuda.synchronize(dev)
@@ -270,10 +295,7 @@ def run_ours(args, w):
 
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
-    stage_ms = {name: statistics.mean(ev[a].elapsed_time(ev[b]) for ev in stage)
-                for name, a, b in (("absorb", 0, 1), ("attention", 1, 2), ("combine", 2, 3), ("upproj", 3, 4))}
-    if sess.appends:
-        stage_ms["append"] = statistics.mean(s.elapsed_time(ev[0]) for s, ev in zip(starts, stage))
+    stage_ms = {k: v / K for k, v in stage_acc.items()}
     max_total_ms = mdist.max_over_ranks(total_ms, dev)
     value = mdist.throughput(sb["total"] * K, ws, max_total_ms / 1e3) / 1e9
 
@@ -334,6 +356,7 @@ def run_ours(args, w):
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / K},
         "gpu_launches": K * sess.kernels_per_step(),
+        "timed_as": "eager API calls" if args.no_graph else "CUDA graph replay of one decode step per timed step",
         "clocks": clk.summary(),
         "step_bytes": sb,
     }
@@ -357,6 +380,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of as a graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

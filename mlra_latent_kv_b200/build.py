@@ -48,26 +48,31 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, out: str | None = None, defines=()) -> str:
+    """Builds the library (``out`` and ``defines`` select a separately named
+    variant, e.g. one with -DMLRA_TRACE pipeline tracing)."""
+    lib = out or LIB
+    if not force and out is None and up_to_date():
         return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    bdir = BUILD_DIR if out is None else BUILD_DIR + "_" + os.path.basename(out).replace(".", "_")
+    os.makedirs(bdir, exist_ok=True)
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-dc", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-I", os.path.join(ROOT, "include"), "-dc", src,
+               "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
            *objs, "-o", tmp, "-lcuda"]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -39,6 +39,7 @@
 #include <mutex>
 
 #include "attn_tc.h"
+#include "host_cache.h"
 #include "ptx.cuh"
 
 namespace mlra {
@@ -46,47 +47,129 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 192;             // warp 0: TMA, warp 1: MMA, warps 2-5: softmax
+// warp 0: TMA, warp 1: MMA, then 4 softmax warps per branch a CTA owns (one
+// warpgroup covers the 128 TMEM lanes = heads)
+template <int kBrPerCta>
+constexpr int threads_of() { return 64 + 128 * kBrPerCta; }
 constexpr int kQSlotBytes = 128 * 128;    // 128 query rows x 64 bf16
 constexpr int kTileSlotBytes = 64 * 128;  // 64 tokens x 64 bf16
-constexpr int kSlots = 5;                 // 4 latent blocks of 64 dims + the rope block
+constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kXBytes = 64 * 128 * 4;     // one page of fp32 partial scores, 128 rows
+constexpr int kXBytes = 64 * 128 * 2;     // one page of fp16 partial scores, 128 rows
 constexpr float kRescaleLog2 = 8.f;
+// TMEM columns: O [0, 256), then a ring of S buffers of 64 columns per branch
+// the CTA owns: four buffers with one branch per CTA, two with two.
+template <int kBrPerCta>
+constexpr int s_bufs() { return kBrPerCta == 1 ? 4 : 2; }
 
 struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t stage_full[3], stage_empty[3];
-  uint64_t s_full[2], p_full[2];
-  uint64_t pv_done, o_free;
-  uint64_t x_full, x_empty;
+  uint64_t stage_full[kMaxStages], stage_empty[kMaxStages];
+  uint64_t rope_full[2], rope_empty[2];  // MLA: the rope half has its own two-slot ring
+  uint64_t s_full[4], p_full[4], pv_done[4];
+  uint64_t o_free;
+  uint64_t x_full[4], x_empty[4];  // MLA exchange, per lane quarter (one softmax warp each)
   WorkerPlan plan;
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// Shared-memory layout.
+//  MLA (kExch): 4 latent blocks of this CTA's 256 dims per page in a ring of 4
+//  stages; the CTA's half of the rope dims (32, 64-byte swizzle) in its own
+//  two-slot ring, released as soon as QK^T has read it; one fp16 exchange
+//  buffer for the partial scores of one page.
+//  MLRA: 4 latent blocks + the full rope block (128-byte swizzle) per stage,
+//  ring of 3 stages.
 template <bool kExch>
 struct Layout {
-  static constexpr int kStages = kExch ? 2 : 3;
+  static constexpr int kStages = kExch ? 4 : 3;
+  static constexpr int kRopeQBytes = kExch ? 128 * 64 : kQSlotBytes;
+  static constexpr int kRopeTileBytes = kExch ? 64 * 64 : kTileSlotBytes;
+  static constexpr int kRopeRowBytes = kExch ? 64 : 128;
+  static constexpr int kStageBytes = 4 * kTileSlotBytes + (kExch ? 0 : kRopeTileBytes);
   static constexpr int kQ = 0;
-  static constexpr int kTile = kSlots * kQSlotBytes;
-  static constexpr int kX = kTile + kStages * kSlots * kTileSlotBytes;
+  static constexpr int kQRope = 4 * kQSlotBytes;
+  static constexpr int kTile = kQRope + kRopeQBytes;
+  static constexpr int kRope = kTile + kStages * kStageBytes;  // MLA rope ring
+  static constexpr int kX = kRope + (kExch ? 2 * kRopeTileBytes : 0);
   static constexpr int kBars = kX + (kExch ? kXBytes : 0);
   static constexpr int kBytes = kBars + (int)sizeof(Bars) + 1024;  // + alignment slack
+  static_assert(kStageBytes % 1024 == 0 && kTile % 1024 == 0 && kRope % 1024 == 0, "aligned slots");
+  static_assert(kBytes <= 232448, "shared memory");
 };
 
+// Optional pipeline trace (builds with -DMLRA_TRACE only): globaltimer stamps
+// of each role's events for the first kTracePages pages of CTAs 0 and 1.
+#ifdef MLRA_TRACE
+constexpr int kTracePages = 64;
+constexpr int kTraceEvents = 12;
+__device__ unsigned long long g_trace[2][kTracePages][kTraceEvents];
+enum { kEvTma = 0, kEvStageSeen, kEvQkIssued, kEvSReady, kEvSent, kEvRecv, kEvPReady, kEvPvIssued, kEvMath,
+       kEvSoftmaxDone, kEvQkStart, kEvRecvAdded };
+#define MLRA_TRACE_EV(gg, ev)                                                                  \
+  do {                                                                                         \
+    if (blockIdx.x < 2 && (gg) < (uint32_t)kTracePages) g_trace[blockIdx.x][gg][ev] = globaltimer_ns(); \
+  } while (0)
+#else
+#define MLRA_TRACE_EV(gg, ev) \
+  do {                        \
+  } while (0)
+#endif
+
 // wait-site codes recorded with a timeout
-enum { kSiteQEmpty = 1, kSiteStageEmpty, kSiteQFull, kSiteStageFull, kSitePFull, kSiteOFree, kSiteSFull,
-       kSiteXEmpty, kSiteXFull, kSitePvDone };
+enum { kSiteQEmpty = 1, kSiteStageEmpty, kSiteQFull, kSiteMma, kSiteOFree, kSiteSFull, kSiteXEmpty, kSiteXFull,
+       kSitePvDone };
+
+// One page of online softmax for one row (head) in the log2 domain (the
+// queries arrive pre-multiplied by softmax_scale*log2(e), so the scores are
+// base-2 logits).  s: scores in, exp2(s - m) out; tokens >= valid are masked.
+// Returns whether O must be rescaled by corr (the running max grew by more
+// than 2^8); the first page of a piece starts the running state.
+__device__ __forceinline__ bool softmax_page(float (&s)[64], int valid, bool first, float& m_run, float& l_run,
+                                             float& corr) {
+  if (valid < 64) {
+#pragma unroll
+    for (int n = 0; n < 64; ++n)
+      if (n >= valid) s[n] = -INFINITY;
+  }
+  float m8[8];
+#pragma unroll
+  for (int n = 0; n < 64; ++n) m8[n & 7] = (n < 8) ? s[n] : fmaxf(m8[n & 7], s[n]);
+  const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+  bool rescale = false;
+  float m_use;
+  if (first) {
+    m_use = mx;
+    corr = 0.f;
+  } else if (mx > m_run + kRescaleLog2) {
+    m_use = mx;
+    corr = ex2(m_run - mx);
+    rescale = true;
+  } else {
+    m_use = m_run;
+    corr = 1.f;
+  }
+  float a8[8];
+#pragma unroll
+  for (int n = 0; n < 64; ++n) {
+    s[n] = ex2(s[n] - m_use);
+    a8[n & 7] = (n < 8) ? s[n] : a8[n & 7] + s[n];
+  }
+  const float sum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+  l_run = l_run * corr + sum;
+  m_run = m_use;
+  return rescale;
+}
 
 template <bool kExch, int kBrPerCta>
-__global__ void __launch_bounds__(kThreads, 1)
-    attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lat,
-                     const __grid_constant__ CUtensorMap tm_rope, const int* __restrict__ page_table,
-                     const int* __restrict__ seq_lens, float* __restrict__ o_part, float* __restrict__ ml_part,
-                     int* __restrict__ err, AttnArgs a) {
+__global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rope,
+                     const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
+                     const int* __restrict__ page_table, const int* __restrict__ seq_lens,
+                     float* __restrict__ o_part, float* __restrict__ ml_part, int* __restrict__ err, AttnArgs a) {
   using L = Layout<kExch>;
-  constexpr int kStages = L::kStages;
   constexpr int kLatPerBr = 4 / kBrPerCta;      // latent slots per branch
   constexpr int kPvN = 256 / kBrPerCta;         // PV output columns per branch
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
@@ -95,33 +178,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::kQ;
+  uint8_t* sQRope = smem + L::kQRope;
   uint8_t* sTile = smem + L::kTile;
+  uint8_t* sRope = smem + L::kRope;
   uint8_t* sX = smem + L::kX;
+  constexpr int kStages = L::kStages;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::kBars);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = kExch ? cluster_ctarank() : (blockIdx.x & 1u);
   const int c = blockIdx.x >> 1;
-  const bool has_rope = kExch ? (rank == 0) : true;
-  const int n_slots = has_rope ? 5 : 4;
   const int maxL = a.maxp * kPage;
+  const int rope_q_bytes = a.H * (kExch ? 64 : 128);  // H query rows of the rope block
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
     mbar_init(smem_u32(&bars->q_empty), 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&bars->stage_full[s]), 1);
       mbar_init(smem_u32(&bars->stage_empty[s]), 1);
     }
     for (int k = 0; k < 2; ++k) {
-      mbar_init(smem_u32(&bars->s_full[k]), 1);
-      mbar_init(smem_u32(&bars->p_full[k]), 4);
+      mbar_init(smem_u32(&bars->rope_full[k]), 1);
+      mbar_init(smem_u32(&bars->rope_empty[k]), 1);
     }
-    mbar_init(smem_u32(&bars->pv_done), 1);
-    mbar_init(smem_u32(&bars->o_free), 4);
-    mbar_init(smem_u32(&bars->x_full), 128);
-    mbar_init(smem_u32(&bars->x_empty), 128);
+    for (int k = 0; k < 4; ++k) {
+      mbar_init(smem_u32(&bars->s_full[k]), 1);
+      mbar_init(smem_u32(&bars->p_full[k]), 4 * kBrPerCta);
+      mbar_init(smem_u32(&bars->pv_done[k]), 1);
+    }
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(smem_u32(&bars->x_full[q]), 1);
+      mbar_init(smem_u32(&bars->x_empty[q]), 1);
+    }
+    mbar_init(smem_u32(&bars->o_free), 4 * kBrPerCta);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -146,7 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   const WorkerPlan plan = bars->plan;
 
-  auto S_col = [](uint32_t buf, int i) -> uint32_t { return 256u + buf * 128u + (uint32_t)i * 64u; };
+  // S ring (kSB buffers of 64 columns per branch) after the 256 columns of O
+  constexpr int kSB = s_bufs<kBrPerCta>();
+  auto S_col = [](uint32_t buf, int i) -> uint32_t {
+    return 256u + buf * (64u * kBrPerCta) + (uint32_t)i * 64u;
+  };
+  static_assert(256 + kSB * 64 * kBrPerCta <= 512, "TMEM columns overflow");
   auto O_col = [](int i) -> uint32_t { return (uint32_t)i * (uint32_t)kPvN; };
 
   if (warp == 0) {
@@ -155,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_lat);
       tma_prefetch_desc(&tm_rope);
+      if (kExch) tma_prefetch_desc(&tm_q_rope);
       SegWalk walk(plan, a.B, maxL);
       int seg = 0;
       uint32_t g = 0;
@@ -162,10 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && walk.next(seq_lens)) {
         if (seg > 0 && !mbar_wait(smem_u32(&bars->q_empty), (seg - 1) & 1, abort_flag, err, kSiteQEmpty)) break;
         const uint32_t qb = smem_u32(&bars->q_full);
-        mbar_expect_tx(qb, n_slots * kQSlotBytes);
+        mbar_expect_tx(qb, 4 * a.H * 128 + rope_q_bytes);
         for (int s = 0; s < 4; ++s)
-          tma_load_2d(smem_u32(sQ + s * kQSlotBytes), &tm_q, qb, 64 * (4 * (int)rank + s), walk.b * 128);
-        if (has_rope) tma_load_2d(smem_u32(sQ + 4 * kQSlotBytes), &tm_q, qb, a.d_c, walk.b * 128);
+          tma_load_2d(smem_u32(sQ + s * kQSlotBytes), &tm_q, qb, 64 * (4 * (int)rank + s), walk.b * a.H);
+        if (kExch)
+          tma_load_2d(smem_u32(sQRope), &tm_q_rope, qb, a.d_c + 32 * (int)rank, walk.b * a.H);
+        else
+          tma_load_2d(smem_u32(sQRope), &tm_q, qb, a.d_c, walk.b * a.H);
         for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
           const uint32_t st = g % kStages, use = g / kStages;
           if (use > 0 && !mbar_wait(smem_u32(&bars->stage_empty[st]), (use - 1) & 1, abort_flag, err,
@@ -173,246 +273,372 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (kExch && g >= 2 &&
+              !mbar_wait(smem_u32(&bars->rope_empty[g & 1]), ((g >> 1) - 1) & 1, abort_flag, err, kSiteStageEmpty)) {
+            ok = false;
+            break;
+          }
           const int pg = page_of(page_table, a.maxp, a.num_pages, walk.b, p * kPage, err);
           const uint32_t fb = smem_u32(&bars->stage_full[st]);
-          uint8_t* tile = sTile + st * (kSlots * kTileSlotBytes);
-          mbar_expect_tx(fb, n_slots * kTileSlotBytes);
+          uint8_t* tile = sTile + st * L::kStageBytes;
+          mbar_expect_tx(fb, L::kStageBytes);
           for (int s = 0; s < 4; ++s)
             tma_load_2d(smem_u32(tile + s * kTileSlotBytes), &tm_lat, fb, 64 * (4 * (int)rank + s), pg * kPage);
-          if (has_rope) tma_load_2d(smem_u32(tile + 4 * kTileSlotBytes), &tm_rope, fb, 0, pg * kPage);
+          if (kExch) {
+            const uint32_t rb = smem_u32(&bars->rope_full[g & 1]);
+            mbar_expect_tx(rb, L::kRopeTileBytes);
+            tma_load_2d(smem_u32(sRope + (g & 1) * L::kRopeTileBytes), &tm_rope, rb, 32 * (int)rank, pg * kPage);
+          } else {
+            tma_load_2d(smem_u32(tile + 4 * kTileSlotBytes), &tm_rope, fb, 0, pg * kPage);
+          }
+          MLRA_TRACE_EV(g, kEvTma);
         }
         ++seg;
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
+    // Event loop: QK^T of the next landed page and PV of the next page whose P
+    // is ready are issued in whichever order they become possible (QK(g) may
+    // run once PV(g - kSB) is issued: S buffer g % kSB holds P(g - kSB) until then).
     SegWalk walk(plan, a.B, maxL);
     int seg = 0;
     uint32_t g = 0;
     bool ok = true;
-    auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-      if (first && seg > 0 &&
-          !mbar_wait_warp(smem_u32(&bars->o_free), (seg - 1) & 1, abort_flag, err, kSiteOFree))
-        return false;
-      if (!mbar_wait_warp(smem_u32(&bars->p_full[gg & 1]), (gg >> 1) & 1, abort_flag, err, kSitePFull)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t tile = smem_u32(sTile + (gg % kStages) * (kSlots * kTileSlotBytes));
-#pragma unroll
-        for (int i = 0; i < kBrPerCta; ++i) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bd = sdesc_sw128(tile + (i * kLatPerBr) * kTileSlotBytes + ks * 2048, 8192, 1024);
-            mma_ts(tmem + O_col(i), tmem + S_col(gg & 1, i) + 8u * ks, bd, kIdescPV, (first && ks == 0) ? 0u : 1u);
-          }
-        }
-        mma_commit(smem_u32(&bars->stage_empty[gg % kStages]));
-        mma_commit(smem_u32(&bars->pv_done));
-      }
-      __syncwarp();
-      return true;
-    };
+    const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);  // query latent blocks (when read from smem)
+    const uint64_t qrd = kExch ? sdesc_sw64(smem_u32(sQRope), 512) : sdesc_sw128(smem_u32(sQRope), 16, 1024);
     while (ok && walk.next(seq_lens)) {
       if (!mbar_wait_warp(smem_u32(&bars->q_full), seg & 1, abort_flag, err, kSiteQFull)) break;
       tc_fence_after();
-      const uint32_t g0 = g;
-      for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
-        const uint32_t st = g % kStages, use = g / kStages;
-        if (!mbar_wait_warp(smem_u32(&bars->stage_full[st]), use & 1, abort_flag, err, kSiteStageFull)) {
-          ok = false;
-          break;
-        }
-        uint8_t* tile = sTile + st * (kSlots * kTileSlotBytes);
-        const int valid = min(kPage, walk.L - p * kPage);
-        if (valid < kPage) {  // zero the rows past the end of the sequence
-          const int nrow = kPage - valid;
-          const uint4 z = make_uint4(0, 0, 0, 0);
-          for (int idx = lane; idx < nrow * 8 * n_slots; idx += 32) {
-            const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
-            *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+      const uint32_t g0 = g, g_end = g + (uint32_t)(walk.pg1 - walk.pg0);
+      uint32_t g_qk = g0, g_pv = g0;
+      bool o_ready = (seg == 0);
+      long long t_idle = 0;
+      while (g_pv < g_end) {
+        bool progressed = false;
+        if (g_pv < g_qk) {
+          if (!o_ready) {  // the previous piece's O must be drained before the first PV overwrites it
+            bool r = lane == 0 ? mbar_test_wait(smem_u32(&bars->o_free), (seg - 1) & 1) : false;
+            o_ready = __shfl_sync(0xffffffffu, r, 0);
           }
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t qa = smem_u32(sQ), ta = smem_u32(tile);
+          if (o_ready) {
+            bool ready =
+                lane == 0 ? mbar_test_wait(smem_u32(&bars->p_full[g_pv % kSB]), (g_pv / kSB) & 1) : false;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (ready) {
+              tc_fence_after();
+              if (lane == 0) {
+                const uint32_t first = g_pv == g0 ? 1u : 0u;
+                // B = the page's latent blocks read MN-major (the value side of the same tile)
+                const uint64_t vd = sdesc_sw128(smem_u32(sTile + (g_pv % kStages) * L::kStageBytes), 8192, 1024);
+                const uint32_t p_base = tmem + S_col(g_pv % kSB, 0);
 #pragma unroll
-          for (int i = 0; i < kBrPerCta; ++i) {
-            uint32_t kk = 0;
-            for (int j = 0; j < kLatPerBr + (has_rope ? 1 : 0); ++j) {
-              const int s = j < kLatPerBr ? i * kLatPerBr + j : 4;
+                for (int i = 0; i < kBrPerCta; ++i) {
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks, ++kk) {
-                const uint64_t ad = sdesc_sw128(qa + s * kQSlotBytes + ks * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(ta + s * kTileSlotBytes + ks * 32, 16, 1024);
-                mma_ss(tmem + S_col(g & 1, i), ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+                  for (int ks = 0; ks < 4; ++ks)
+                    mma_ts(tmem + O_col(i), p_base + 64u * i + 8u * ks,
+                           vd + (uint64_t)(((i * kLatPerBr) * kTileSlotBytes + ks * 2048) >> 4), kIdescPV,
+                           ks == 0 ? (first ^ 1u) : 1u);
+                }
+                mma_commit(smem_u32(&bars->stage_empty[g_pv % kStages]));
+                mma_commit(smem_u32(&bars->pv_done[g_pv % kSB]));
+                MLRA_TRACE_EV(g_pv, kEvPvIssued);
               }
+              __syncwarp();
+              ++g_pv;
+              progressed = true;
             }
           }
-          mma_commit(smem_u32(&bars->s_full[g & 1]));
         }
-        __syncwarp();
-        if (g > g0 && !issue_pv(g - 1, g - 1 == g0)) {
-          ok = false;
-          break;
+        // QK(g) needs S buffer g % kSB, free once PV(g - kSB) is issued; look
+        // ahead at most two pages past the next PV so that PVs (which free the
+        // stages) are not queued behind a run of QKs
+        if (!progressed && g_qk < g_end && g_qk < g_pv + kSB && g_qk <= g_pv + 2) {
+          const uint32_t st = g_qk % kStages;
+          bool ready = lane == 0 ? mbar_test_wait(smem_u32(&bars->stage_full[st]), (g_qk / kStages) & 1) &&
+                                       (!kExch || mbar_test_wait(smem_u32(&bars->rope_full[g_qk & 1]),
+                                                                 (g_qk >> 1) & 1))
+                                 : false;
+          ready = __shfl_sync(0xffffffffu, ready, 0);
+          if (ready) {
+            if (lane == 0) MLRA_TRACE_EV(g_qk, kEvStageSeen);
+            uint8_t* tile = sTile + st * L::kStageBytes;
+            uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + 4 * kTileSlotBytes;
+            const int p = walk.pg0 + (int)(g_qk - g0);
+            const int valid = min(kPage, walk.L - p * kPage);
+            if (valid < kPage) {  // zero the rows past the end of the sequence
+              const int nrow = kPage - valid;
+              const uint4 z = make_uint4(0, 0, 0, 0);
+              for (int idx = lane; idx < nrow * 8 * 4; idx += 32) {
+                const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
+                *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+              }
+              constexpr int kRopeChunks = L::kRopeRowBytes / 16;
+              for (int idx = lane; idx < nrow * kRopeChunks; idx += 32)
+                *reinterpret_cast<uint4*>(rope_tile + (valid + idx / kRopeChunks) * L::kRopeRowBytes +
+                                          (idx % kRopeChunks) * 16) = z;
+              fence_proxy_async_smem();
+            }
+            __syncwarp();
+            tc_fence_after();
+            if (lane == 0) {
+              MLRA_TRACE_EV(g_qk, kEvQkStart);
+              // descriptors = per-stage base + compile-time offsets (no per-MMA rebuild)
+              const uint64_t td = sdesc_sw128(smem_u32(tile), 16, 1024);
+              const uint32_t s_base = tmem + S_col(g_qk % kSB, 0);
+#pragma unroll
+              for (int i = 0; i < kBrPerCta; ++i) {
+#pragma unroll
+                for (int j = 0; j < kLatPerBr; ++j) {
+                  const int s = i * kLatPerBr + j;
+#pragma unroll
+                  for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t bd = td + (uint64_t)((s * kTileSlotBytes + ks * 32) >> 4);
+                    mma_ss(s_base + 64u * i, qd + (uint64_t)((s * kQSlotBytes + ks * 32) >> 4), bd, kIdescQK,
+                           (j | ks) ? 1u : 0u);
+                  }
+                }
+                if (kExch) {
+                  const uint64_t trd = sdesc_sw64(smem_u32(rope_tile), 512);
+#pragma unroll
+                  for (int ks = 0; ks < 2; ++ks)
+                    mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2), trd + (uint64_t)(ks * 2), kIdescQK, 1u);
+                } else {
+#pragma unroll
+                  for (int ks = 0; ks < 4; ++ks)
+                    mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2),
+                           td + (uint64_t)((4 * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
+                }
+              }
+              mma_commit(smem_u32(&bars->s_full[g_qk % kSB]));
+              if (kExch) mma_commit(smem_u32(&bars->rope_empty[g_qk & 1]));
+              MLRA_TRACE_EV(g_qk, kEvQkIssued);
+              if (g_qk + 1 == g_end) mma_commit(smem_u32(&bars->q_empty));  // last read of this Q
+            }
+            __syncwarp();
+            ++g_qk;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_idle = 0;
+        } else {
+          __nanosleep(32);  // idle: leave issue slots to the softmax warp sharing this sub-partition
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          if (t_idle == 0) t_idle = clock64();
+          if (clock64() - t_idle > kWaitCycles) {
+            if (lane == 0) {
+              *abort_flag = 1;
+              report_error(err, kErrTimeout, kSiteMma, (int)blockIdx.x);
+            }
+            ok = false;
+            break;
+          }
         }
       }
-      if (!ok || g == g0) break;
-      if (!issue_pv(g - 1, g - 1 == g0)) break;
-      if (lane == 0) mma_commit(smem_u32(&bars->q_empty));
-      __syncwarp();
+      ok = __all_sync(0xffffffffu, ok);
+      g = g_end;
       ++seg;
     }
   } else {
     // -------------------------------------------------------------- softmax
     const int q4 = warp & 3;
+    const int bi = (warp - 2) >> 2;  // branch of this warpgroup (0 unless 2 branches per CTA)
     const int row = q4 * 32 + lane;  // head
+    const bool real = row < a.H;
+    const bool warp_real = q4 * 32 < a.H;  // warp-uniform: some lane holds a real head
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t peer = rank ^ 1u;
-    const uint32_t x_remote = kExch ? map_to_cta(smem_u32(sX), peer) : 0u;
-    const uint32_t xfull_remote = kExch ? map_to_cta(smem_u32(&bars->x_full), peer) : 0u;
-    const uint32_t xempty_remote = kExch ? map_to_cta(smem_u32(&bars->x_empty), peer) : 0u;
     SegWalk walk(plan, a.B, maxL);
     uint32_t g = 0;
     bool ok = true;
-    while (ok && walk.next(seq_lens)) {
-      const uint32_t g0 = g;
-      float m_run[kBrPerCta], l_run[kBrPerCta];
+
+    // MLA only.  Each softmax warp exchanges its 32 rows with the same warp of
+    // the peer CTA through its own barriers, so no warp waits for another.
+    const int q_rows = a.H - q4 * 32 < 0 ? 0 : (a.H - q4 * 32 > 32 ? 32 : a.H - q4 * 32);
+    // send my fp16 partial scores of page gg to the peer's buffer gg & 1
+    // (one buffer: the peer's page gg goes in only after my rows of page gg-1
+    // were read; the receive-then-send order below keeps that deadlock-free)
+    auto send_partial = [&](uint32_t gg, const uint32_t (&own_h)[32]) -> bool {
+      if (gg > 0 && !mbar_wait_warp<true>(smem_u32(&bars->x_empty[q4]), (gg - 1) & 1, abort_flag, err,
+                                          kSiteXEmpty))
+        return false;
+      if (real) {
+        const uint32_t dst = map_to_cta(smem_u32(sX), peer);
+        const uint32_t bar = map_to_cta(smem_u32(&bars->x_full[q4]), peer);
 #pragma unroll
-      for (int i = 0; i < kBrPerCta; ++i) {
-        m_run[i] = -INFINITY;
-        l_run[i] = 0.f;
+        for (int q = 0; q < 8; ++q)
+          st_async_v4(dst + (uint32_t)((q * 128 + row) * 16), own_h[4 * q], own_h[4 * q + 1], own_h[4 * q + 2],
+                      own_h[4 * q + 3], bar);
       }
-      for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
-        const int valid = min(kPage, walk.L - p * kPage);
-        if (!mbar_wait_warp(smem_u32(&bars->s_full[g & 1]), (g >> 1) & 1, abort_flag, err, kSiteSFull)) {
-          ok = false;
-          break;
+      if (lane == 0) {
+        mbar_expect_tx(smem_u32(&bars->x_full[q4]), (uint32_t)q_rows * 128u);
+        if (row == 0) MLRA_TRACE_EV(gg, kEvSent);
+      }
+      return true;
+    };
+    // s = f16(own) + f16(peer) for page gg, identical bits on both CTAs
+    auto receive_partial = [&](uint32_t gg, float (&s)[64], const uint32_t (&own_h)[32]) -> bool {
+      if (!mbar_wait_warp<true>(smem_u32(&bars->x_full[q4]), gg & 1, abort_flag, err, kSiteXFull)) return false;
+      if (row == 0) MLRA_TRACE_EV(gg, kEvRecv);
+      if (real) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sX + (q * 128 + row) * 16);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 mine = unpack_f16x2(own_h[4 * q + j]);
+            const float2 theirs = unpack_f16x2(w[j]);
+            s[8 * q + 2 * j] = mine.x + theirs.x;
+            s[8 * q + 2 * j + 1] = mine.y + theirs.y;
+          }
         }
-        tc_fence_after();
-        uint32_t P[kBrPerCta][32];
-        float corr[kBrPerCta];
+      }
+      if (row == 0) MLRA_TRACE_EV(gg, kEvRecvAdded);
+      // my rows of the buffer are read: the peer warp may refill them
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_cta(smem_u32(&bars->x_empty[q4]), peer));
+      return true;
+    };
+    auto load_scores = [&](uint32_t gg, float (&s)[64]) -> bool {
+      if (!mbar_wait_warp(smem_u32(&bars->s_full[gg % kSB]), (gg / kSB) & 1, abort_flag, err, kSiteSFull))
+        return false;
+      tc_fence_after();
+      if (row == 0) MLRA_TRACE_EV(gg, kEvSReady);
+      if (warp_real) {
+        uint32_t lo[32], hi[32];
+        tmem_ld32x2(tmem + lane_off + S_col(gg % kSB, bi), tmem + lane_off + S_col(gg % kSB, bi) + 32u, lo, hi);
+#pragma unroll
+        for (int n = 0; n < 32; ++n) {
+          s[n] = __uint_as_float(lo[n]);
+          s[n + 32] = __uint_as_float(hi[n]);
+        }
+      }
+      return true;
+    };
+
+    while (ok && walk.next(seq_lens)) {
+      const uint32_t g0 = g, g_end = g + (uint32_t)(walk.pg1 - walk.pg0);
+      float m_run = -INFINITY, l_run = 0.f;
+      float cur[64];
+      uint32_t cur_h[32], nxt_h[32];  // MLA: my partial scores as sent (fp16 pairs)
+      auto load_pack_send = [&](uint32_t gg, uint32_t (&h)[32]) -> bool {
+        if (!load_scores(gg, cur)) return false;
+        if (!warp_real) return true;  // padding rows only: nothing to exchange
+#pragma unroll
+        for (int j = 0; j < 32; ++j) h[j] = pack_f16x2(cur[2 * j], cur[2 * j + 1]);
+        return send_partial(gg, h);
+      };
+      if (kExch) {
+        if (!load_pack_send(g, cur_h)) break;
+      } else if (!load_scores(g, cur)) {
+        break;
+      }
+      for (; g < g_end; ++g) {
+        const int valid = min(kPage, walk.L - (walk.pg0 + (int)(g - g0)) * kPage);
+        if (kExch) {
+          // receive this page first (its buffer release then orders only
+          // remote writes issued a page ago), then send the next page's
+          // partial so that it travels during this page's softmax
+          if (warp_real && !receive_partial(g, cur, cur_h)) {
+            ok = false;
+            break;
+          }
+          if (g + 1 < g_end) {
+            float tmp[64];
+            if (!load_scores(g + 1, tmp)) {
+              ok = false;
+              break;
+            }
+            if (warp_real) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) nxt_h[j] = pack_f16x2(tmp[2 * j], tmp[2 * j + 1]);
+              if (!send_partial(g + 1, nxt_h)) {
+                ok = false;
+                break;
+              }
+            }
+          }
+        } else if (g > g0) {
+          if (!load_scores(g, cur)) {
+            ok = false;
+            break;
+          }
+        }
+        uint32_t P[32];
+        float corr = 1.f;
         bool rescale = false;
+        if (warp_real) {
+          rescale = softmax_page(cur, valid, g == g0, m_run, l_run, corr);
+          if (row == 0) MLRA_TRACE_EV(g, kEvSoftmaxDone);
 #pragma unroll
-        for (int i = 0; i < kBrPerCta; ++i) {
-          uint32_t lo[32], hi[32];
-          tmem_ld32(tmem + lane_off + S_col(g & 1, i), lo);
-          tmem_ld32(tmem + lane_off + S_col(g & 1, i) + 32u, hi);
-          if (kExch) {
-            // send my partial scores to the peer, receive and add its partial
-            if (g > 0 && !mbar_wait_warp<true>(smem_u32(&bars->x_empty), (g - 1) & 1, abort_flag, err, kSiteXEmpty)) {
-              ok = false;
-              break;
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              st_cluster_v4(x_remote + (uint32_t)((q * 128 + row) * 16), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2],
-                            lo[4 * q + 3]);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              st_cluster_v4(x_remote + (uint32_t)(((8 + q) * 128 + row) * 16), hi[4 * q], hi[4 * q + 1],
-                            hi[4 * q + 2], hi[4 * q + 3]);
-            mbar_arrive_cluster(xfull_remote);
-            if (!mbar_wait_warp<true>(smem_u32(&bars->x_full), g & 1, abort_flag, err, kSiteXFull)) {
-              ok = false;
-              break;
-            }
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float4 v = *reinterpret_cast<const float4*>(sX + (q * 128 + row) * 16);
-              uint32_t* d = q < 8 ? &lo[4 * q] : &hi[4 * (q - 8)];
-              d[0] = __float_as_uint(__uint_as_float(d[0]) + v.x);
-              d[1] = __float_as_uint(__uint_as_float(d[1]) + v.y);
-              d[2] = __float_as_uint(__uint_as_float(d[2]) + v.z);
-              d[3] = __float_as_uint(__uint_as_float(d[3]) + v.w);
-            }
-            mbar_arrive_cluster(xempty_remote);
-          }
-          // online softmax over this page (log2 domain)
-          float s[64];
-          float mx = -INFINITY;
-#pragma unroll
-          for (int n = 0; n < 64; ++n) {
-            const float raw = __uint_as_float(n < 32 ? lo[n] : hi[n - 32]);
-            s[n] = n < valid ? raw * a.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, s[n]);
-          }
-          float m_use;
-          if (g == g0) {
-            m_use = mx;
-            corr[i] = 0.f;
-          } else if (mx > m_run[i] + kRescaleLog2) {
-            m_use = mx;
-            corr[i] = ex2(m_run[i] - mx);
-            rescale = true;
-          } else {
-            m_use = m_run[i];
-            corr[i] = 1.f;
-          }
-          float sum = 0.f;
-#pragma unroll
-          for (int n = 0; n < 64; ++n) {
-            s[n] = ex2(s[n] - m_use);
-            sum += s[n];
-          }
-          l_run[i] = l_run[i] * corr[i] + sum;
-          m_run[i] = m_use;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) P[i][j] = pack_bf16x2(s[2 * j], s[2 * j + 1]);
+          for (int j = 0; j < 32; ++j) P[j] = pack_bf16x2(cur[2 * j], cur[2 * j + 1]);
         }
-        if (!ok) break;
-        if (g > g0) {
-          if (!mbar_wait_warp(smem_u32(&bars->pv_done), (g - 1) & 1, abort_flag, err, kSitePvDone)) {
+        if (row == 0) MLRA_TRACE_EV(g, kEvMath);
+        // O is rescaled only when the running max jumped; that needs PV(g-1)
+        // complete.  PV(g-1) signals pv_done[(g-1) % kSB]; that barrier is at
+        // most one phase from this target (PV(g-1-kSB) finished before QK(g-1),
+        // whose scores were read, and PV(g-1+kSB) needs a P not yet written),
+        // so its parity identifies PV(g-1) without waiting on every page.
+        if (g > g0 && warp_real && __any_sync(0xffffffffu, rescale)) {
+          if (!mbar_wait_warp(smem_u32(&bars->pv_done[(g - 1) % kSB]), ((g - 1) / kSB) & 1, abort_flag, err,
+                              kSitePvDone)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
+          {
+            for (int cc = 0; cc < kPvN; cc += 32) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_off + O_col(bi) + cc, o);
 #pragma unroll
-            for (int i = 0; i < kBrPerCta; ++i) {
-              for (int cc = 0; cc < kPvN; cc += 32) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_off + O_col(i) + cc, o);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr[i]);
-                tmem_st32(tmem + lane_off + O_col(i) + cc, o);
-              }
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+              tmem_st32(tmem + lane_off + O_col(bi) + cc, o);
             }
           }
         }
-#pragma unroll
-        for (int i = 0; i < kBrPerCta; ++i) tmem_st32(tmem + lane_off + S_col(g & 1, i), P[i]);
+        if (warp_real) tmem_st32(tmem + lane_off + S_col(g % kSB, bi), P);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[g & 1]));
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[g % kSB]));
+        if (row == 0) MLRA_TRACE_EV(g, kEvPReady);
+        if (kExch) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) cur_h[j] = nxt_h[j];
+        }
       }
-      if (!ok || g == g0) break;
+      if (!ok) break;
       // epilogue: O and (m, l) of this piece to its slot
-      if (!mbar_wait_warp(smem_u32(&bars->pv_done), (g - 1) & 1, abort_flag, err, kSitePvDone)) break;
+      if (!mbar_wait_warp(smem_u32(&bars->pv_done[(g - 1) % kSB]), ((g - 1) / kSB) & 1, abort_flag, err,
+                          kSitePvDone))
+        break;
       tc_fence_after();
       const int slot = c + walk.b;
-      const bool real = row < a.H;
-#pragma unroll
-      for (int i = 0; i < kBrPerCta; ++i) {
+      if (warp_real) {
         for (int cc = 0; cc < kPvN; cc += 32) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + O_col(i) + cc, o);
+          tmem_ld32(tmem + lane_off + O_col(bi) + cc, o);
           if (real) {
-            const int d0 = 256 * (int)rank + (int)O_col(i) + cc;
+            const int d0 = 256 * (int)rank + (int)O_col(bi) + cc;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int d = d0 + 4 * q;
-              float4 v = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
-                                     __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
-              *reinterpret_cast<float4*>(o_part + (((size_t)slot * (a.d_c / 4) + d / 4) * a.H + row) * 4) = v;
+            for (int q = 0; q < 4; ++q) {
+              const int d = d0 + 8 * q;
+              float4* dst = reinterpret_cast<float4*>(o_part + (((size_t)slot * (a.d_c / 8) + d / 8) * a.H + row) * 8);
+              dst[0] = make_float4(__uint_as_float(o[8 * q]), __uint_as_float(o[8 * q + 1]),
+                                   __uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
+              dst[1] = make_float4(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]),
+                                   __uint_as_float(o[8 * q + 6]), __uint_as_float(o[8 * q + 7]));
             }
           }
         }
         if (real && (!kExch || rank == 0)) {
-          const int br = kExch ? 0 : (int)rank * kBrPerCta + i;
-          ml_part[(((size_t)slot * a.n_branch + br) * 2 + 0) * a.H + row] = m_run[i];
-          ml_part[(((size_t)slot * a.n_branch + br) * 2 + 1) * a.H + row] = l_run[i];
+          const int br = kExch ? 0 : (int)rank * kBrPerCta + bi;
+          ml_part[(((size_t)slot * a.n_branch + br) * 2 + 0) * a.H + row] = m_run;
+          ml_part[(((size_t)slot * a.n_branch + br) * 2 + 1) * a.H + row] = l_run;
         }
       }
       tc_fence_before();
@@ -431,42 +657,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-cudaError_t get_encoder() {
-  std::call_once(g_encode_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return g_encode ? cudaSuccess : cudaErrorNotSupported;
-}
-
-// 2-D bf16 map over rows x cols (cols contiguous), box = box_cols x box_rows, 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <bool kExch, int kBrPerCta>
-cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tl, const CUtensorMap& tr, const int* page_table,
+cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tl, const CUtensorMap& tr,
+                           const int* page_table,
                            const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                            cudaStream_t st) {
   auto kern = attend_tc_kernel<kExch, kBrPerCta>;
   const int smem = Layout<kExch>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.G, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads_of<kBrPerCta>(), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -476,7 +678,7 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tl, const C
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tq, tl, tr, page_table, seq_lens, o_part, ml_part, err, a);
+  return cudaLaunchKernelEx(&cfg, kern, tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a);
 }
 
 }  // namespace
@@ -489,21 +691,35 @@ bool tc_supported(int dtype, int H, int d_c, int d_r, int n_branch, int /*d_h*/,
 cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop, const int* page_table,
                              const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                              cudaStream_t st) {
-  cudaError_t e = get_encoder();
-  if (e != cudaSuccess) return e;
-  CUtensorMap tq, tl, tr;
-  if (!make_map(&tq, q_ws, (uint64_t)(a.d_c + a.d_r), (uint64_t)a.B * kTcHeads, 64, 128) ||
-      !make_map(&tl, lat, (uint64_t)a.d_c, (uint64_t)a.num_pages * kPage, 64, 64) ||
-      !make_map(&tr, rop, (uint64_t)a.d_r, (uint64_t)a.num_pages * kPage, 64, 64))
+  CUtensorMap tq, tqr, tl, tr;
+  const bool exch = a.n_branch == 1;
+  if (!tmap_2d(&tq, q_ws, (uint64_t)(a.d_c + a.d_r), (uint64_t)a.B * a.H, 64, (uint32_t)a.H) ||
+      !tmap_2d(&tl, lat, (uint64_t)a.d_c, (uint64_t)a.num_pages * kPage, 64, 64))
     return cudaErrorInvalidValue;
+  if (exch) {  // each CTA of the pair takes half of the rope dims
+    if (!tmap_2d_sw64(&tqr, q_ws, (uint64_t)(a.d_c + a.d_r), (uint64_t)a.B * a.H, 32, (uint32_t)a.H) ||
+        !tmap_2d_sw64(&tr, rop, (uint64_t)a.d_r, (uint64_t)a.num_pages * kPage, 32, 64))
+      return cudaErrorInvalidValue;
+  } else {
+    tqr = tq;
+    if (!tmap_2d(&tr, rop, (uint64_t)a.d_r, (uint64_t)a.num_pages * kPage, 64, 64)) return cudaErrorInvalidValue;
+  }
   switch (a.n_branch) {
-    case 1: return launch_variant<true, 1>(tq, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
-    case 2: return launch_variant<false, 1>(tq, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
-    case 4: return launch_variant<false, 2>(tq, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
+    case 1: return launch_variant<true, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
+    case 2: return launch_variant<false, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
+    case 4: return launch_variant<false, 2>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-void tc_shutdown() {}
+void tc_shutdown() { host_cache_clear(); }
+
+#ifdef MLRA_TRACE
+// Copies the pipeline trace of the last attention launch (trace builds only).
+extern "C" __attribute__((visibility("default"))) int mlra_trace_read(unsigned long long* host, size_t n) {
+  const size_t bytes = sizeof(g_trace) < n * sizeof(unsigned long long) ? sizeof(g_trace) : n * sizeof(unsigned long long);
+  return (int)cudaMemcpyFromSymbol(host, g_trace, bytes);
+}
+#endif
 
 }  // namespace mlra

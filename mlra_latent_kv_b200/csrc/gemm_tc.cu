@@ -1,0 +1,347 @@
+// tcgen05 kernels for the two small per-head contractions of the decode step
+// (yololab.net, "超越 GQA 的推理革命…", section "矩陣吸收": W_UK is folded into
+// the query before attention and W_UV applied after it):
+//
+//   a2  q_lat[b, h, :] = q_nope[b, h, :] . W_UK[h]        (+ RoPE of q_rope)
+//   a4+a5  o_lat[b, h, :] = combine of the split-KV partials of (b, h)
+//          out[b, h, :]   = o_lat[b, h, :] . W_UV[h]
+//
+// Both are weight-bandwidth bound (every weight is read once per step and used
+// for B rows), so they run "swap-AB": the weight is the M x K operand (M =
+// latent or value dims, MN-major straight from its row-major layout by TMA),
+// the batch is N (padded to a multiple of 16 with TMA zero fill), and one CTA
+// per (head, 128-row M tile) streams its weight slice once.  The combine is
+// fused into the up-projection: the CTA of head h merges the partials of every
+// sequence into bf16 rows of the MMA's B operand in shared memory, so o_lat
+// never goes to HBM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm_tc.h"
+#include "host_cache.h"
+#include "ptx.cuh"
+
+namespace mlra {
+namespace {
+
+using namespace ptx;
+
+// 128-byte-swizzled K-major tile of `rows` rows x 64 bf16: byte offset of the
+// 16-byte chunk (row, chunk) -- the layout TMA writes and the MMA reads.
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t tmem_cols_for(int n) {
+  uint32_t c = 32;
+  while ((int)c < n) c <<= 1;
+  return c;
+}
+
+// ---------------------------------------------------------------------------
+// a2: query absorption.  grid (H, d_c / 128), block 128.
+//   A (M = 128 latent dims, K = d_h) = W_UK[h][:, m0:m0+128]   MN-major
+//   B (N = Bp batch rows, K = d_h)   = q_nope[:, h, :]          K-major
+//   D (TMEM, 128 lanes x Bp)         -> q_ws[b][h][m0 + lane] (bf16)
+// Block (h, 0) also rotates q_rope[:, h] into q_ws[b][h][d_c:].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128, 1)
+    absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                     const __nv_bfloat16* __restrict__ q_rope, const int* __restrict__ q_pos,
+                     __nv_bfloat16* __restrict__ q_ws, int* __restrict__ err, GemmArgs a, RopeTable tab) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int a_bytes = 2 * a.K * 128;          // two 64-column M blocks of K rows
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + a_bytes;               // K/64 blocks of Bp rows
+  __shared__ uint64_t full_bar, done_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int h = blockIdx.x, m0 = blockIdx.y * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = tmem_cols_for(a.Bp);
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&full_bar), 1);
+    mbar_init(smem_u32(&done_bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_base), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    const uint32_t fb = smem_u32(&full_bar);
+    mbar_expect_tx(fb, a_bytes + (a.K / 64) * a.Bp * 128);
+    for (int mb = 0; mb < 2; ++mb) tma_load_2d(smem_u32(sA + mb * a.K * 128), &tm_w, fb, m0 + 64 * mb, h * a.K);
+    for (int kb = 0; kb < a.K / 64; ++kb) tma_load_3d(smem_u32(sB + kb * a.Bp * 128), &tm_q, fb, 64 * kb, h, 0);
+    ok = mbar_wait(fb, 0, &abort_flag, err, 20);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, a.Bp, true, false);
+      const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
+      const uint64_t bd0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+      const uint64_t bkb = (uint64_t)((a.Bp * 128) >> 4);
+      for (int kb = 0; kb < a.K / 64; ++kb) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss(tmem, ad0 + (uint64_t)(kb * 4 + ks) * 128u, bd0 + kb * bkb + (uint64_t)(ks * 2), idesc,
+                 (kb | ks) ? 1u : 0u);
+      }
+      mma_commit(smem_u32(&done_bar));
+    }
+  }
+  // RoPE of the query (independent of the MMA)
+  if (blockIdx.y == 0) {
+    const int pairs = a.d_r / 2;
+    for (int idx = threadIdx.x; idx < a.B * pairs; idx += blockDim.x) {
+      const int b = idx / pairs, i = idx % pairs;
+      const __nv_bfloat16* src = q_rope + ((size_t)b * a.H + h) * a.d_r + 2 * i;
+      const float x0 = __bfloat162float(src[0]), x1 = __bfloat162float(src[1]);
+      float s, c;
+      rope_sincos(tab, i, __ldg(q_pos + b), &s, &c);
+      __nv_bfloat16* dst = q_ws + ((size_t)b * a.H + h) * (a.d_c + a.d_r) + a.d_c + 2 * i;
+      dst[0] = __float2bfloat16_rn((x0 * c - x1 * s) * a.q_scale);
+      dst[1] = __float2bfloat16_rn((x0 * s + x1 * c) * a.q_scale);
+    }
+  }
+  if (mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 21)) {
+    tc_fence_after();
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    for (int cc = 0; cc < a.Bp; cc += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + cc, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int b = cc + j;
+        if (b < a.B)
+          q_ws[((size_t)b * a.H + h) * (a.d_c + a.d_r) + m0 + warp * 32 + lane] =
+              __float2bfloat16_rn(__uint_as_float(v[j]) * a.q_scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+// ---------------------------------------------------------------------------
+// a4 + a5: split combine fused into the output up-projection.
+// grid (H, d_v / 128), block 256.
+//   A (M = 128 value dims, K = d_c) = W_UV[h][:, m0:m0+128]   MN-major (TMA)
+//   B (N = Bp batch rows, K = d_c)  = o_lat[:, h, :] built here in smem:
+//       o_lat[b, h, br cols] = branch_scale * sum_s 2^(m_s - M) o_s / L
+//   D (TMEM, 128 lanes x Bp)        -> out[b][h][m0 + lane] (bf16)
+// ---------------------------------------------------------------------------
+constexpr int kCuThreads = 256;
+
+__global__ void __launch_bounds__(kCuThreads, 1)
+    combine_upproj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ o_part,
+                             const float* __restrict__ ml_part, const int* __restrict__ seq_lens,
+                             __nv_bfloat16* __restrict__ out, int* __restrict__ err, GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int a_bytes = 2 * a.K * 128;             // K = d_c rows, two 64-column M blocks
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + a_bytes;                  // d_c/64 blocks of Bp rows
+  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * a.Bp * 128);  // [slots][n_branch]
+  int* s_c0 = reinterpret_cast<int*>(s_wt + (size_t)(a.G + a.B) * a.n_branch);
+  int* s_c1 = s_c0 + a.B;
+  __shared__ uint64_t full_bar, done_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  __shared__ long long s_T;
+  const int h = blockIdx.x, m0 = blockIdx.y * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = tmem_cols_for(a.Bp);
+  const int maxL = a.maxp * kPage;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&full_bar), 1);
+    mbar_init(smem_u32(&done_bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_base), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  if (threadIdx.x == 0) {  // stream the weight slice while the combine runs
+    const uint32_t fb = smem_u32(&full_bar);
+    mbar_expect_tx(fb, a_bytes);
+    const int box_rows = a.K < 256 ? a.K : 256;
+    for (int mb = 0; mb < 2; ++mb)
+      for (int r = 0; r < a.K; r += box_rows)
+        tma_load_2d(smem_u32(sA + mb * a.K * 128 + r * 128), &tm_w, fb, m0 + 64 * mb, h * a.K + r);
+  }
+  // sequence -> worker range (the split plan of the attention kernel)
+  if (warp == 0) {
+    long long T = 0;
+    for (int base = 0; base < a.B; base += 32) {
+      const int np = base + lane < a.B ? npages_of(seq_len_at(seq_lens, base + lane, maxL)) : 0;
+      T += warp_sum_i(np);
+    }
+    long long prefix = 0;
+    for (int base = 0; base < a.B; base += 32) {
+      const int b = base + lane;
+      const int np = b < a.B ? npages_of(seq_len_at(seq_lens, b, maxL)) : 0;
+      const int incl = warp_incl_scan(np);
+      if (b < a.B) {
+        const long long P = prefix + incl - np;
+        s_c0[b] = np > 0 ? worker_of_page(P, T, a.G) : 0;
+        s_c1[b] = np > 0 ? worker_of_page(P + np - 1, T, a.G) : -1;
+      }
+      prefix += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_T = T;
+  }
+  __syncthreads();
+  const long long T = s_T;
+  // per (b, branch): weights of the pieces
+  for (int idx = threadIdx.x; idx < a.B * a.n_branch; idx += blockDim.x) {
+    const int b = idx / a.n_branch, br = idx % a.n_branch;
+    const int c0 = s_c0[b], c1 = s_c1[b];
+    float M = -INFINITY;
+    for (int c = c0; c <= c1; ++c)
+      if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G))
+        M = fmaxf(M, ml_part[(((size_t)(c + b) * a.n_branch + br) * 2 + 0) * a.H + h]);
+    float Lsum = 0.f;
+    for (int c = c0; c <= c1; ++c)
+      if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G)) {
+        const size_t base = ((size_t)(c + b) * a.n_branch + br) * 2;
+        Lsum += exp2f(ml_part[(base + 0) * a.H + h] - M) * ml_part[(base + 1) * a.H + h];
+      }
+    const float scale = a.branch_scale / Lsum;
+    for (int c = c0; c <= c1; ++c) {
+      const bool nonempty = worker_start(c, T, a.G) != worker_start(c + 1, T, a.G);
+      s_wt[(size_t)(c + b) * a.n_branch + br] =
+          nonempty ? exp2f(ml_part[(((size_t)(c + b) * a.n_branch + br) * 2 + 0) * a.H + h] - M) * scale : 0.f;
+    }
+  }
+  __syncthreads();
+  // o_lat rows (bf16) straight into the swizzled B operand; padding rows are zero
+  const int chunks = a.K / 8;
+  const int d_cb = a.K / a.n_branch;
+  for (int idx = threadIdx.x; idx < a.Bp * chunks; idx += blockDim.x) {
+    const int b = idx / chunks, ch = idx % chunks;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    if (b < a.B) {
+      const int br = (ch * 8) / d_cb;
+      for (int c = s_c0[b]; c <= s_c1[b]; ++c) {
+        const float w = s_wt[(size_t)(c + b) * a.n_branch + br];
+        if (w == 0.f) continue;
+        const float4* src = reinterpret_cast<const float4*>(o_part + (((size_t)(c + b) * chunks + ch) * a.H + h) * 8);
+        const float4 u = src[0], v = src[1];
+        acc[0] = fmaf(w, u.x, acc[0]);
+        acc[1] = fmaf(w, u.y, acc[1]);
+        acc[2] = fmaf(w, u.z, acc[2]);
+        acc[3] = fmaf(w, u.w, acc[3]);
+        acc[4] = fmaf(w, v.x, acc[4]);
+        acc[5] = fmaf(w, v.y, acc[5]);
+        acc[6] = fmaf(w, v.z, acc[6]);
+        acc[7] = fmaf(w, v.w, acc[7]);
+      }
+    }
+    uint4 pk;
+    pk.x = pack_bf16x2(acc[0], acc[1]);
+    pk.y = pack_bf16x2(acc[2], acc[3]);
+    pk.z = pack_bf16x2(acc[4], acc[5]);
+    pk.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(sB + (ch / 8) * a.Bp * 128 + sw128_off(b, ch % 8)) = pk;
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (mbar_wait(smem_u32(&full_bar), 0, &abort_flag, err, 22)) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, a.Bp, true, false);
+      const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
+      const uint64_t bd0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+      const uint64_t bkb = (uint64_t)((a.Bp * 128) >> 4);
+      for (int kb = 0; kb < a.K / 64; ++kb) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss(tmem, ad0 + (uint64_t)(kb * 4 + ks) * 128u, bd0 + kb * bkb + (uint64_t)(ks * 2), idesc,
+                 (kb | ks) ? 1u : 0u);
+      }
+      mma_commit(smem_u32(&done_bar));
+    }
+  }
+  if (warp < 4 && mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 23)) {
+    tc_fence_after();
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    for (int cc = 0; cc < a.Bp; cc += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + cc, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int b = cc + j;
+        if (b < a.B)
+          out[((size_t)b * a.H + h) * a.N_out + m0 + warp * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+}  // namespace
+
+bool absorb_tc_supported(int dtype, int B, int d_h, int d_c) {
+  return dtype == 1 && B >= 1 && B <= 256 && d_h % 64 == 0 && d_h <= 256 && d_c % 128 == 0;
+}
+
+// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B) plus d_c/64 x Bp x 128 B of o_lat rows
+bool upproj_tc_supported(int dtype, int B, int d_c, int d_v) {
+  return dtype == 1 && B >= 1 && B <= 96 && d_c % 64 == 0 && d_c <= 512 && (d_c <= 256 || d_c % 256 == 0) &&
+         d_v % 128 == 0;
+}
+
+int batch_pad(int B) { return B <= 16 ? 16 : (B + 15) / 16 * 16; }
+
+cudaError_t launch_absorb_tc(const void* q_nope, const void* q_rope, const int* q_pos, const void* W_UK, void* q_ws,
+                             int* err, const GemmArgs& a, const RopeTable& tab, cudaStream_t st) {
+  CUtensorMap tw, tq;
+  if (!tmap_2d(&tw, W_UK, (uint64_t)a.d_c, (uint64_t)a.H * a.K, 64, (uint32_t)a.K) ||
+      !tmap_3d_batch(&tq, q_nope, (uint64_t)a.K, (uint64_t)a.H, (uint64_t)a.B, (uint32_t)a.Bp))
+    return cudaErrorInvalidValue;
+  const int smem = 1024 + 2 * a.K * 128 + (a.K / 64) * a.Bp * 128;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(absorb_tc_kernel), smem);
+  if (e != cudaSuccess) return e;
+  absorb_tc_kernel<<<dim3(a.H, a.d_c / 128), 128, smem, st>>>(tw, tq, (const __nv_bfloat16*)q_rope, q_pos,
+                                                              (__nv_bfloat16*)q_ws, err, a, tab);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_upproj_tc(const float* o_part, const float* ml_part, const int* seq_lens, const void* W_UV,
+                                     void* out, int* err, const GemmArgs& a, cudaStream_t st) {
+  CUtensorMap tw;
+  if (!tmap_2d(&tw, W_UV, (uint64_t)a.N_out, (uint64_t)a.H * a.K, 64, (uint32_t)(a.K < 256 ? a.K : 256)))
+    return cudaErrorInvalidValue;
+  const int smem = 1024 + 2 * a.K * 128 + (a.K / 64) * a.Bp * 128 + (a.G + a.B) * a.n_branch * 4 + 2 * a.B * 4;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(combine_upproj_tc_kernel), smem);
+  if (e != cudaSuccess) return e;
+  combine_upproj_tc_kernel<<<dim3(a.H, a.N_out / 128), kCuThreads, smem, st>>>(
+      tw, o_part, ml_part, seq_lens, (__nv_bfloat16*)out, err, a);
+  return cudaGetLastError();
+}
+
+}  // namespace mlra

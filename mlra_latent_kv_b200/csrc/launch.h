@@ -10,6 +10,7 @@ namespace mlra {
 
 struct AbsorbArgs {
   int B, H, Hq, d_h, d_c, d_r;
+  float q_scale;  // multiplies q_lat and the rotated q_rope (1 unless the attention kernel expects pre-scaled queries)
 };
 
 struct AttnArgs {

@@ -8,6 +8,8 @@
 
 #include "../../include/mlra.h"
 #include "attn_tc.h"
+#include "gemm_tc.h"
+#include "host_cache.h"
 #include "launch.h"
 
 using namespace mlra;
@@ -113,7 +115,7 @@ mlra_status make_plan(const mlra_dims* d, DecodePlan* p) {
     G = p->tc ? sms / 2 : sms;
   }
   p->G = G;
-  p->Hq = p->tc ? kTcHeads : d->H;
+  p->Hq = d->H;
   const size_t qe = p->tc ? 2 : 4;
   const size_t slots = (size_t)G + d->B - 1;
   size_t off = kErrBytes;
@@ -160,14 +162,27 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
   const RopeTable tab = rope_table(d);
   cudaError_t e;
 
-  if (ev && ev[0]) cudaEventRecord(ev[0], stream);
-  AbsorbArgs aa{d->B, d->H, p.Hq, d->d_h, d->d_c, d->d_r};
-  e = launch_absorb(d->dtype, p.tc, q_nope, q_rope, q_pos, W_UK, q_ws, aa, tab, stream);
+  const bool tc_absorb = p.tc && absorb_tc_supported(d->dtype, d->B, d->d_h, d->d_c);
+  const bool tc_upproj = p.tc && upproj_tc_supported(d->dtype, d->B, d->d_c, d->d_v);
+  // The tcgen05 attention kernel takes queries pre-multiplied by scale*log2(e)
+  // (its scores are then base-2 logits directly); the CUDA-core kernel scales itself.
+  const float scale_log2 = scale_of(d) * 1.4426950408889634f;
+  const float q_scale = p.tc ? scale_log2 : 1.0f;
+  GemmArgs ga{d->B, batch_pad(d->B), d->H, d->d_h, d->d_c, d->d_r, d->d_v, p.G, d->n_branch,
+              d->max_pages_per_seq, branch_scale, q_scale};
+
+  if (ev) record_event(ev[0], stream);
+  if (tc_absorb) {
+    e = launch_absorb_tc(q_nope, q_rope, q_pos, W_UK, q_ws, err, ga, tab, stream);
+  } else {
+    AbsorbArgs aa{d->B, d->H, p.Hq, d->d_h, d->d_c, d->d_r, q_scale};
+    e = launch_absorb(d->dtype, p.tc, q_nope, q_rope, q_pos, W_UK, q_ws, aa, tab, stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "absorb launch");
-  if (ev && ev[1]) cudaEventRecord(ev[1], stream);
+  if (ev) record_event(ev[1], stream);
 
   AttnArgs at{d->B, d->H, d->d_c, d->d_r, d->n_branch, d->max_pages_per_seq, d->num_pages, p.G,
-              scale_of(d) * 1.4426950408889634f};
+              p.tc ? 1.0f : scale_log2};
   if (p.tc) {
     e = launch_attend_tc(q_ws, latent_cache, rope_cache, page_table, seq_lens, o_part, ml_part, err, at, stream);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 attention launch");
@@ -176,17 +191,24 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
                            o_part, ml_part, err, at, stream);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   }
-  if (ev && ev[2]) cudaEventRecord(ev[2], stream);
+  if (ev) record_event(ev[2], stream);
 
-  CombineArgs ca{d->B, d->H, d->d_c, d->n_branch, p.G, d->max_pages_per_seq, branch_scale};
-  e = launch_combine(p.tc, o_part, ml_part, seq_lens, o_lat, ca, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-  if (ev && ev[3]) cudaEventRecord(ev[3], stream);
-
-  UpArgs ua{d->B, d->H, d->d_c, d->d_v};
-  e = launch_upproj(d->dtype, p.tc, o_lat, W_UV, out, ua, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "up-projection launch");
-  if (ev && ev[4]) cudaEventRecord(ev[4], stream);
+  if (tc_upproj) {  // combine fused into the up-projection: stage 3 is empty
+    if (ev) record_event(ev[3], stream);
+    GemmArgs gu = ga;
+    gu.K = d->d_c;
+    e = launch_combine_upproj_tc(o_part, ml_part, seq_lens, W_UV, out, err, gu, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine + up-projection launch");
+  } else {
+    CombineArgs ca{d->B, d->H, d->d_c, d->n_branch, p.G, d->max_pages_per_seq, branch_scale};
+    e = launch_combine(p.tc, o_part, ml_part, seq_lens, o_lat, ca, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    if (ev) record_event(ev[3], stream);
+    UpArgs ua{d->B, d->H, d->d_c, d->d_v};
+    e = launch_upproj(d->dtype, p.tc, o_lat, W_UV, out, ua, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "up-projection launch");
+  }
+  if (ev) record_event(ev[4], stream);
   return MLRA_OK;
 }
 

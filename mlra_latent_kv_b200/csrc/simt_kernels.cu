@@ -38,8 +38,8 @@ __global__ void __launch_bounds__(128) absorb_kernel(const T* __restrict__ q_nop
       float x0 = to_f(src[0]), x1 = to_f(src[1]);
       float s, c;
       rope_sincos(tab, i, __ldg(q_pos + b), &s, &c);
-      dst[0] = from_f<QO>(x0 * c - x1 * s);
-      dst[1] = from_f<QO>(x0 * s + x1 * c);
+      dst[0] = from_f<QO>((x0 * c - x1 * s) * a.q_scale);
+      dst[1] = from_f<QO>((x0 * s + x1 * c) * a.q_scale);
     }
     return;
   }
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(128) absorb_kernel(const T* __restrict__ q_nop
       }
 #pragma unroll
       for (int i = 0; i < kAbsorbB; ++i)
-        if (i < nb) q_ws[((size_t)(b0 + i) * a.Hq + h) * row + col] = from_f<QO>(acc[i]);
+        if (i < nb) q_ws[((size_t)(b0 + i) * a.Hq + h) * row + col] = from_f<QO>(acc[i] * a.q_scale);
     }
     __syncthreads();
   }
@@ -79,7 +79,10 @@ __global__ void __launch_bounds__(128) absorb_kernel(const T* __restrict__ q_nop
 // block stages kTileTok cache rows (latent | rope) in shared memory as fp32.
 // Lane l owns latent dims l + 32k and rope dims l + 32k.
 // Writes the unnormalised partial o (relative to the running max m, in log2
-// units) and m, l per branch to slot c + b.
+// units) and m, l per branch to slot c + b.  Partial layout (shared with the
+// tcgen05 kernels): o_part[slot][d_c/8][H][8] fp32 (32-byte chunks, so a head
+// per thread writes and a head per block reads whole sectors),
+// ml_part[slot][n_branch][2][H] (m, l).
 // ---------------------------------------------------------------------------
 constexpr int kTileTok = 16;
 constexpr int kMaxDpl = 16;  // d_c <= 512
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(const float* __restric
       for (int k = 0; k < kMaxDpl; ++k) {
         if (k < dpl) {
           const int d = lane + 32 * k;
-          o_part[(((size_t)slot * (a.d_c / 4) + d / 4) * a.H + h) * 4 + (d & 3)] = o[k];
+          o_part[(((size_t)slot * (a.d_c / 8) + d / 8) * a.H + h) * 8 + (d & 7)] = o[k];
         }
       }
       if (lane == 0) {
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
         if (MLRA_WORKER_EMPTY(c)) continue;
         const size_t base = ((size_t)(c + b) * a.n_branch + br) * 2;
         const float w = exp2f(ml_part[(base + 0) * a.H + h] - M);
-        acc = fmaf(w, o_part[(((size_t)(c + b) * (a.d_c / 4) + d / 4) * a.H + h) * 4 + (d & 3)], acc);
+        acc = fmaf(w, o_part[(((size_t)(c + b) * (a.d_c / 8) + d / 8) * a.H + h) * 8 + (d & 7)], acc);
       }
       dst[d] = from_f<OT>(acc * inv);
     }

@@ -106,4 +106,11 @@ class DecodeSession:
             abi.check_status(self.app_ws)
 
     def kernels_per_step(self) -> int:
-        return 4 + (2 if self.appends else 0)
+        """Kernels one step launches: append (2, when it appends), absorption,
+        attention, and combine + up-projection (one fused tcgen05 kernel, or two
+        CUDA-core kernels), following the library's kernel choice."""
+        w = self.w
+        tc = (self.dims.kernel != 1 and w.dtype == "bf16" and w.d_c == 512 and w.d_r == 64 and w.H <= 128
+              and w.n_branch in (1, 2, 4))
+        fused = tc and w.B <= 96 and w.d_v % 128 == 0
+        return (2 if self.appends else 0) + 2 + (1 if fused else 2)

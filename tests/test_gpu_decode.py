@@ -48,6 +48,16 @@ def test_reduced_workloads(name, kernel):
     assert err <= tol, f"{name}/{kernel}: max err {err:.3e} > tol {tol:.3e} (rel l2 {rel_l2(out, ref):.2e})"
 
 
+@pytest.mark.parametrize("G", [1, 2, 5])
+@pytest.mark.parametrize("name", [n for n in REDUCED if n != "tiny_mla_fp32"])
+def test_reduced_workloads_few_workers(name, G):
+    """Few split workers, so every worker runs many pages and several sequences
+    back to back (stage ring wrap-around, S double buffer, piece changes)."""
+    w = synth.workload(name).with_(**REDUCED[name])
+    err, tol, out, ref, _ = run_case(w, "auto", num_splits=G)
+    assert err <= tol, f"{name}/G={G}: max err {err:.3e} > tol {tol:.3e}"
+
+
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("H", [128, 64, 32, 8])
 def test_edge_lengths_mla(H, kernel):
