@@ -49,14 +49,15 @@ using namespace ptx;
 
 // warp 0: TMA, warp 1: MMA, then 4 softmax warps per branch a CTA owns (one
 // warpgroup covers the 128 TMEM lanes = heads)
-template <int kBrPerCta>
-constexpr int threads_of() { return 64 + 128 * kBrPerCta; }
+template <bool kExch, int kBrPerCta>
+constexpr int threads_of() { return 64 + 128 * kBrPerCta + (kExch ? 128 : 0); }  // + MLA exchange warps
 constexpr int kQSlotBytes = 128 * 128;    // 128 query rows x 64 bf16
 constexpr int kTileSlotBytes = 64 * 128;  // 64 tokens x 64 bf16
 constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kXBytes = 64 * 128 * 2;     // one page of fp16 partial scores, 128 rows
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kPrefetch = 8;              // pages warmed in L2 ahead of the TMA ring
 // TMEM columns: O [0, 256), then a ring of S buffers of 64 columns per branch
 // the CTA owns: four buffers with one branch per CTA, two with two.
 template <int kBrPerCta>
@@ -69,6 +70,7 @@ struct Bars {
   uint64_t s_full[4], p_full[4], pv_done[4];
   uint64_t o_free;
   uint64_t x_full[4], x_empty[4];  // MLA exchange, per lane quarter (one softmax warp each)
+  uint64_t xs_read[4][4];          // MLA: the exchange warp of a quarter has read S buffer k
   WorkerPlan plan;
   uint32_t tmem_base;
   int abort_flag;
@@ -164,7 +166,7 @@ __device__ __forceinline__ bool softmax_page(float (&s)[64], int valid, bool fir
 }
 
 template <bool kExch, int kBrPerCta>
-__global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
+__global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rope,
                      const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
                      const int* __restrict__ page_table, const int* __restrict__ seq_lens,
@@ -211,8 +213,12 @@ __global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
     for (int q = 0; q < 4; ++q) {
       mbar_init(smem_u32(&bars->x_full[q]), 1);
       mbar_init(smem_u32(&bars->x_empty[q]), 1);
+      for (int k = 0; k < 4; ++k) mbar_init(smem_u32(&bars->xs_read[q][k]), 1);
     }
     mbar_init(smem_u32(&bars->o_free), 4 * kBrPerCta);
+    // MLA: the peer's partial scores of page 0 are expected in phase 0 of x_full
+    if (kExch)
+      for (int q = 0; q * 32 < a.H; ++q) mbar_expect_tx(smem_u32(&bars->x_full[q]), (uint32_t)min(32, a.H - q * 32) * 128u);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -253,6 +259,25 @@ __global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
       tma_prefetch_desc(&tm_rope);
       if (kExch) tma_prefetch_desc(&tm_q_rope);
       SegWalk walk(plan, a.B, maxL);
+      // A second cursor runs kPrefetch pages ahead and warms L2 with each page,
+      // so that a ring refill waits for L2 rather than for HBM latency.
+      SegWalk pf(plan, a.B, maxL);
+      int pf_p = 0;
+      bool pf_live = pf.next(seq_lens);
+      if (pf_live) pf_p = pf.pg0;
+      auto prefetch_one = [&]() {
+        if (!pf_live) return;
+        const int pg = __ldg(page_table + (size_t)pf.b * a.maxp + pf_p);
+        if (pg >= 0 && pg < a.num_pages) {  // an invalid id is reported by the load itself
+          for (int s = 0; s < 4; ++s) tma_prefetch_l2_2d(&tm_lat, 64 * (4 * (int)rank + s), pg * kPage);
+          tma_prefetch_l2_2d(&tm_rope, kExch ? 32 * (int)rank : 0, pg * kPage);
+        }
+        if (++pf_p >= pf.pg1) {
+          pf_live = pf.next(seq_lens);
+          if (pf_live) pf_p = pf.pg0;
+        }
+      };
+      for (int k = 0; k < kPrefetch; ++k) prefetch_one();
       int seg = 0;
       uint32_t g = 0;
       bool ok = true;
@@ -267,6 +292,7 @@ __global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
         else
           tma_load_2d(smem_u32(sQRope), &tm_q, qb, a.d_c, walk.b * a.H);
         for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
+          prefetch_one();
           const uint32_t st = g % kStages, use = g / kStages;
           if (use > 0 && !mbar_wait(smem_u32(&bars->stage_empty[st]), (use - 1) & 1, abort_flag, err,
                                     kSiteStageEmpty)) {
@@ -443,6 +469,58 @@ __global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
       g = g_end;
       ++seg;
     }
+  } else if (kExch && warp >= 6) {
+    // ------------------------------------------------------------- exchange
+    // MLA: send this CTA's partial scores of every page (fp16, its 32 rows)
+    // to the same warp of the peer CTA as soon as QK^T has produced them.
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const bool real = row < a.H;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t peer = rank ^ 1u;
+    if (q4 * 32 < a.H) {
+      const uint32_t dst = map_to_cta(smem_u32(sX), peer);
+      const uint32_t bar = map_to_cta(smem_u32(&bars->x_full[q4]), peer);
+      SegWalk walk(plan, a.B, maxL);
+      uint32_t g = 0;
+      bool ok = true;
+      while (ok && walk.next(seq_lens)) {
+        for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
+          if (!mbar_wait_warp(smem_u32(&bars->s_full[g % kSB]), (g / kSB) & 1, abort_flag, err, kSiteSFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t lo[32], hi[32];
+          tmem_ld32x2(tmem + lane_off + S_col(g % kSB, 0), tmem + lane_off + S_col(g % kSB, 0) + 32u, lo, hi);
+          tc_fence_before();
+          __syncwarp();
+          // S(g) may now be overwritten by P(g).  One barrier per S buffer: the
+          // softmax warp's wait for page g then sees at most one phase ahead
+          // (page g + kSB needs QK(g + kSB), hence P(g) written).
+          if (lane == 0) mbar_arrive(smem_u32(&bars->xs_read[q4][g % kSB]));
+          uint32_t h[32];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            h[j] = pack_f16x2(__uint_as_float(lo[2 * j]), __uint_as_float(lo[2 * j + 1]));
+            h[16 + j] = pack_f16x2(__uint_as_float(hi[2 * j]), __uint_as_float(hi[2 * j + 1]));
+          }
+          // single buffer: the peer warp must have read my page g-1
+          if (g > 0 && !mbar_wait_warp<true>(smem_u32(&bars->x_empty[q4]), (g - 1) & 1, abort_flag, err,
+                                             kSiteXEmpty)) {
+            ok = false;
+            break;
+          }
+          if (real) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              st_async_v4(dst + (uint32_t)((q * 128 + row) * 16), h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3],
+                          bar);
+          }
+          if (row == 0) MLRA_TRACE_EV(g, kEvSent);
+        }
+      }
+    }
   } else {
     // -------------------------------------------------------------- softmax
     const int q4 = warp & 3;
@@ -452,121 +530,59 @@ __global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
     const bool warp_real = q4 * 32 < a.H;  // warp-uniform: some lane holds a real head
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t peer = rank ^ 1u;
+    const int q_rows = a.H - q4 * 32 < 0 ? 0 : (a.H - q4 * 32 > 32 ? 32 : a.H - q4 * 32);
     SegWalk walk(plan, a.B, maxL);
     uint32_t g = 0;
     bool ok = true;
 
-    // MLA only.  Each softmax warp exchanges its 32 rows with the same warp of
-    // the peer CTA through its own barriers, so no warp waits for another.
-    const int q_rows = a.H - q4 * 32 < 0 ? 0 : (a.H - q4 * 32 > 32 ? 32 : a.H - q4 * 32);
-    // send my fp16 partial scores of page gg to the peer's buffer gg & 1
-    // (one buffer: the peer's page gg goes in only after my rows of page gg-1
-    // were read; the receive-then-send order below keeps that deadlock-free)
-    auto send_partial = [&](uint32_t gg, const uint32_t (&own_h)[32]) -> bool {
-      if (gg > 0 && !mbar_wait_warp<true>(smem_u32(&bars->x_empty[q4]), (gg - 1) & 1, abort_flag, err,
-                                          kSiteXEmpty))
-        return false;
-      if (real) {
-        const uint32_t dst = map_to_cta(smem_u32(sX), peer);
-        const uint32_t bar = map_to_cta(smem_u32(&bars->x_full[q4]), peer);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          st_async_v4(dst + (uint32_t)((q * 128 + row) * 16), own_h[4 * q], own_h[4 * q + 1], own_h[4 * q + 2],
-                      own_h[4 * q + 3], bar);
-      }
-      if (lane == 0) {
-        mbar_expect_tx(smem_u32(&bars->x_full[q4]), (uint32_t)q_rows * 128u);
-        if (row == 0) MLRA_TRACE_EV(gg, kEvSent);
-      }
-      return true;
-    };
-    // s = f16(own) + f16(peer) for page gg, identical bits on both CTAs
-    auto receive_partial = [&](uint32_t gg, float (&s)[64], const uint32_t (&own_h)[32]) -> bool {
-      if (!mbar_wait_warp<true>(smem_u32(&bars->x_full[q4]), gg & 1, abort_flag, err, kSiteXFull)) return false;
-      if (row == 0) MLRA_TRACE_EV(gg, kEvRecv);
-      if (real) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 v = *reinterpret_cast<const uint4*>(sX + (q * 128 + row) * 16);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 mine = unpack_f16x2(own_h[4 * q + j]);
-            const float2 theirs = unpack_f16x2(w[j]);
-            s[8 * q + 2 * j] = mine.x + theirs.x;
-            s[8 * q + 2 * j + 1] = mine.y + theirs.y;
-          }
-        }
-      }
-      if (row == 0) MLRA_TRACE_EV(gg, kEvRecvAdded);
-      // my rows of the buffer are read: the peer warp may refill them
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_cta(smem_u32(&bars->x_empty[q4]), peer));
-      return true;
-    };
-    auto load_scores = [&](uint32_t gg, float (&s)[64]) -> bool {
-      if (!mbar_wait_warp(smem_u32(&bars->s_full[gg % kSB]), (gg / kSB) & 1, abort_flag, err, kSiteSFull))
-        return false;
-      tc_fence_after();
-      if (row == 0) MLRA_TRACE_EV(gg, kEvSReady);
-      if (warp_real) {
-        uint32_t lo[32], hi[32];
-        tmem_ld32x2(tmem + lane_off + S_col(gg % kSB, bi), tmem + lane_off + S_col(gg % kSB, bi) + 32u, lo, hi);
-#pragma unroll
-        for (int n = 0; n < 32; ++n) {
-          s[n] = __uint_as_float(lo[n]);
-          s[n + 32] = __uint_as_float(hi[n]);
-        }
-      }
-      return true;
-    };
-
     while (ok && walk.next(seq_lens)) {
       const uint32_t g0 = g, g_end = g + (uint32_t)(walk.pg1 - walk.pg0);
       float m_run = -INFINITY, l_run = 0.f;
-      float cur[64];
-      uint32_t cur_h[32], nxt_h[32];  // MLA: my partial scores as sent (fp16 pairs)
-      auto load_pack_send = [&](uint32_t gg, uint32_t (&h)[32]) -> bool {
-        if (!load_scores(gg, cur)) return false;
-        if (!warp_real) return true;  // padding rows only: nothing to exchange
-#pragma unroll
-        for (int j = 0; j < 32; ++j) h[j] = pack_f16x2(cur[2 * j], cur[2 * j + 1]);
-        return send_partial(gg, h);
-      };
-      if (kExch) {
-        if (!load_pack_send(g, cur_h)) break;
-      } else if (!load_scores(g, cur)) {
-        break;
-      }
       for (; g < g_end; ++g) {
         const int valid = min(kPage, walk.L - (walk.pg0 + (int)(g - g0)) * kPage);
-        if (kExch) {
-          // receive this page first (its buffer release then orders only
-          // remote writes issued a page ago), then send the next page's
-          // partial so that it travels during this page's softmax
-          if (warp_real && !receive_partial(g, cur, cur_h)) {
+        float cur[64];
+        if (!mbar_wait_warp(smem_u32(&bars->s_full[g % kSB]), (g / kSB) & 1, abort_flag, err, kSiteSFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (row == 0) MLRA_TRACE_EV(g, kEvSReady);
+        if (warp_real) {
+          uint32_t lo[32], hi[32];
+          tmem_ld32x2(tmem + lane_off + S_col(g % kSB, bi), tmem + lane_off + S_col(g % kSB, bi) + 32u, lo, hi);
+#pragma unroll
+          for (int n = 0; n < 32; ++n) {
+            cur[n] = __uint_as_float(lo[n]);
+            cur[n + 32] = __uint_as_float(hi[n]);
+          }
+        }
+        if (kExch && warp_real) {
+          // s = f16(mine) + f16(peer's): the same bits on both CTAs of the pair
+          if (!mbar_wait_warp<true>(smem_u32(&bars->x_full[q4]), g & 1, abort_flag, err, kSiteXFull)) {
             ok = false;
             break;
           }
-          if (g + 1 < g_end) {
-            float tmp[64];
-            if (!load_scores(g + 1, tmp)) {
-              ok = false;
-              break;
-            }
-            if (warp_real) {
+          if (row == 0) MLRA_TRACE_EV(g, kEvRecv);
+          if (real) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) nxt_h[j] = pack_f16x2(tmp[2 * j], tmp[2 * j + 1]);
-              if (!send_partial(g + 1, nxt_h)) {
-                ok = false;
-                break;
+            for (int q = 0; q < 8; ++q) {
+              const uint4 v = *reinterpret_cast<const uint4*>(sX + (q * 128 + row) * 16);
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float2 mine = unpack_f16x2(pack_f16x2(cur[8 * q + 2 * j], cur[8 * q + 2 * j + 1]));
+                const float2 theirs = unpack_f16x2(w[j]);
+                cur[8 * q + 2 * j] = mine.x + theirs.x;
+                cur[8 * q + 2 * j + 1] = mine.y + theirs.y;
               }
             }
           }
-        } else if (g > g0) {
-          if (!load_scores(g, cur)) {
-            ok = false;
-            break;
+          if (row == 0) MLRA_TRACE_EV(g, kEvRecvAdded);
+          // page g consumed: arm the next phase, then let the peer refill the buffer
+          __syncwarp();
+          if (lane == 0) {
+            mbar_expect_tx(smem_u32(&bars->x_full[q4]), (uint32_t)q_rows * 128u);
+            mbar_arrive_cluster(map_to_cta(smem_u32(&bars->x_empty[q4]), peer));
           }
         }
         uint32_t P[32];
@@ -591,25 +607,27 @@ __global__ void __launch_bounds__(threads_of<kBrPerCta>(), 1)
             break;
           }
           tc_fence_after();
-          {
-            for (int cc = 0; cc < kPvN; cc += 32) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_off + O_col(bi) + cc, o);
+          for (int cc = 0; cc < kPvN; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + O_col(bi) + cc, o);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
-              tmem_st32(tmem + lane_off + O_col(bi) + cc, o);
-            }
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+            tmem_st32(tmem + lane_off + O_col(bi) + cc, o);
           }
         }
-        if (warp_real) tmem_st32(tmem + lane_off + S_col(g % kSB, bi), P);
+        if (warp_real) {
+          // MLA: the exchange warp must have read S(g) before P(g) overwrites it
+          if (kExch && !mbar_wait_warp(smem_u32(&bars->xs_read[q4][g % kSB]), (g / kSB) & 1, abort_flag, err,
+                                       kSiteSFull)) {
+            ok = false;
+            break;
+          }
+          tmem_st32(tmem + lane_off + S_col(g % kSB, bi), P);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[g % kSB]));
         if (row == 0) MLRA_TRACE_EV(g, kEvPReady);
-        if (kExch) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) cur_h[j] = nxt_h[j];
-        }
       }
       if (!ok) break;
       // epilogue: O and (m, l) of this piece to its slot
@@ -668,7 +686,7 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const 
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.G, 1, 1);
-  cfg.blockDim = dim3(threads_of<kBrPerCta>(), 1, 1);
+  cfg.blockDim = dim3(threads_of<kExch, kBrPerCta>(), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
