@@ -57,7 +57,9 @@ constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kXBytes = 64 * 128 * 2;     // one page of fp16 partial scores, 128 rows
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kPrefetch = 8;              // pages warmed in L2 ahead of the TMA ring
+constexpr int kIdAhead = 8;               // page ids read this many pages before their tile
+constexpr int kIdRing = 16;
+static_assert(kIdRing >= kIdAhead + 2, "id ring holds the ids in flight");
 // TMEM columns: O [0, 256), then a ring of S buffers of 64 columns per branch
 // the CTA owns: four buffers with one branch per CTA, two with two.
 template <int kBrPerCta>
@@ -72,6 +74,7 @@ struct Bars {
   uint64_t x_full[4], x_empty[4];  // MLA exchange, per lane quarter (one softmax warp each)
   uint64_t xs_read[4][4];          // MLA: the exchange warp of a quarter has read S buffer k
   WorkerPlan plan;
+  int page_ids[16];  // producer's ring of fetched page ids
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -107,6 +110,7 @@ struct Layout {
 constexpr int kTracePages = 64;
 constexpr int kTraceEvents = 12;
 __device__ unsigned long long g_trace[2][kTracePages][kTraceEvents];
+__device__ unsigned long long g_span[1024][2];  // entry and exit stamp of every CTA
 enum { kEvTma = 0, kEvStageSeen, kEvQkIssued, kEvSReady, kEvSent, kEvRecv, kEvPReady, kEvPvIssued, kEvMath,
        kEvSoftmaxDone, kEvQkStart, kEvRecvAdded };
 #define MLRA_TRACE_EV(gg, ev)                                                                  \
@@ -122,6 +126,31 @@ enum { kEvTma = 0, kEvStageSeen, kEvQkIssued, kEvSReady, kEvSent, kEvRecv, kEvPR
 // wait-site codes recorded with a timeout
 enum { kSiteQEmpty = 1, kSiteStageEmpty, kSiteQFull, kSiteMma, kSiteOFree, kSiteSFull, kSiteXEmpty, kSiteXFull,
        kSitePvDone };
+
+// Cursor over a worker's pages in walk order that reads each page's id from
+// the page table (the producer runs one of these ahead of its loads).
+struct IdFetch {
+  SegWalk w;
+  int p;
+  bool live;
+  __device__ __forceinline__ IdFetch(const WorkerPlan& plan, int B, int maxL, const int* seq_lens)
+      : w(plan, B, maxL), p(0), live(false) {
+    live = w.next(seq_lens);
+    if (live) p = w.pg0;
+  }
+  __device__ __forceinline__ void step(const int* seq_lens) {
+    if (++p >= w.pg1) {
+      live = w.next(seq_lens);
+      if (live) p = w.pg0;
+    }
+  }
+  // id of the current page (not yet waited for), then advance
+  __device__ __forceinline__ int fetch(const int* seq_lens, const int* page_table, int maxp) {
+    const int id = __ldg(page_table + (size_t)w.b * maxp + p);
+    step(seq_lens);
+    return id;
+  }
+};
 
 // One page of online softmax for one row (head) in the log2 domain (the
 // queries arrive pre-multiplied by softmax_scale*log2(e), so the scores are
@@ -189,6 +218,10 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dep_launch();  // the combine kernel may set up (and load its weights) as this grid retires
+#ifdef MLRA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_span[blockIdx.x][0] = globaltimer_ns();
+#endif
   const uint32_t rank = kExch ? cluster_ctarank() : (blockIdx.x & 1u);
   const int c = blockIdx.x >> 1;
   const int maxL = a.maxp * kPage;
@@ -253,31 +286,34 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
+    // Page ids are read kIdAhead pages before their tile is loaded (a second
+    // cursor over the same pages) and parked in a small ring, so that no
+    // page-table load sits between a freed stage and its refill.  The first
+    // kIdAhead ids are read by the lanes in parallel; later a fetched id is
+    // written to the ring one page after its load was issued.
+    IdFetch ids(plan, a.B, maxL, seq_lens);
+    {
+      int my_b = -1, my_p = 0;
+      for (int k = 0; k < kIdAhead && ids.live; ++k) {
+        if (lane == k) {
+          my_b = ids.w.b;
+          my_p = ids.p;
+        }
+        ids.step(seq_lens);
+      }
+      if (my_b >= 0) bars->page_ids[lane] = __ldg(page_table + (size_t)my_b * a.maxp + my_p);
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_lat);
       tma_prefetch_desc(&tm_rope);
       if (kExch) tma_prefetch_desc(&tm_q_rope);
+      grid_dep_wait();  // the absorbed queries come from the previous kernel
       SegWalk walk(plan, a.B, maxL);
-      // A second cursor runs kPrefetch pages ahead and warms L2 with each page,
-      // so that a ring refill waits for L2 rather than for HBM latency.
-      SegWalk pf(plan, a.B, maxL);
-      int pf_p = 0;
-      bool pf_live = pf.next(seq_lens);
-      if (pf_live) pf_p = pf.pg0;
-      auto prefetch_one = [&]() {
-        if (!pf_live) return;
-        const int pg = __ldg(page_table + (size_t)pf.b * a.maxp + pf_p);
-        if (pg >= 0 && pg < a.num_pages) {  // an invalid id is reported by the load itself
-          for (int s = 0; s < 4; ++s) tma_prefetch_l2_2d(&tm_lat, 64 * (4 * (int)rank + s), pg * kPage);
-          tma_prefetch_l2_2d(&tm_rope, kExch ? 32 * (int)rank : 0, pg * kPage);
-        }
-        if (++pf_p >= pf.pg1) {
-          pf_live = pf.next(seq_lens);
-          if (pf_live) pf_p = pf.pg0;
-        }
-      };
-      for (int k = 0; k < kPrefetch; ++k) prefetch_one();
+      int* id_ring = bars->page_ids;
+      int pend = 0;
+      bool has_pend = false;
       int seg = 0;
       uint32_t g = 0;
       bool ok = true;
@@ -292,7 +328,9 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
         else
           tma_load_2d(smem_u32(sQRope), &tm_q, qb, a.d_c, walk.b * a.H);
         for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
-          prefetch_one();
+          if (has_pend) id_ring[(g - 1 + kIdAhead) % kIdRing] = pend;
+          has_pend = ids.live;
+          if (has_pend) pend = ids.fetch(seq_lens, page_table, a.maxp);  // the id of page g + kIdAhead
           const uint32_t st = g % kStages, use = g / kStages;
           if (use > 0 && !mbar_wait(smem_u32(&bars->stage_empty[st]), (use - 1) & 1, abort_flag, err,
                                     kSiteStageEmpty)) {
@@ -304,7 +342,11 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
             ok = false;
             break;
           }
-          const int pg = page_of(page_table, a.maxp, a.num_pages, walk.b, p * kPage, err);
+          int pg = id_ring[g % kIdRing];
+          if (pg < 0 || pg >= a.num_pages) {  // reported, and replaced by page 0 so that no load leaves the pool
+            report_error(err, kErrDeviceCheck, walk.b, p * kPage);
+            pg = 0;
+          }
           const uint32_t fb = smem_u32(&bars->stage_full[st]);
           uint8_t* tile = sTile + st * L::kStageBytes;
           mbar_expect_tx(fb, L::kStageBytes);
@@ -670,6 +712,9 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
   if (kExch) cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
+#ifdef MLRA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_span[blockIdx.x][1] = globaltimer_ns();
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -679,7 +724,7 @@ template <bool kExch, int kBrPerCta>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tl, const CUtensorMap& tr,
                            const int* page_table,
                            const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool pdl) {
   auto kern = attend_tc_kernel<kExch, kBrPerCta>;
   const int smem = Layout<kExch>::kBytes;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
@@ -689,13 +734,15 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const 
   cfg.blockDim = dim3(threads_of<kExch, kBrPerCta>(), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kExch ? 2 : 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a);
 }
 
@@ -708,7 +755,7 @@ bool tc_supported(int dtype, int H, int d_c, int d_r, int n_branch, int /*d_h*/,
 
 cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop, const int* page_table,
                              const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool pdl) {
   CUtensorMap tq, tqr, tl, tr;
   const bool exch = a.n_branch == 1;
   if (!tmap_2d(&tq, q_ws, (uint64_t)(a.d_c + a.d_r), (uint64_t)a.B * a.H, 64, (uint32_t)a.H) ||
@@ -723,9 +770,9 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
     if (!tmap_2d(&tr, rop, (uint64_t)a.d_r, (uint64_t)a.num_pages * kPage, 64, 64)) return cudaErrorInvalidValue;
   }
   switch (a.n_branch) {
-    case 1: return launch_variant<true, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
-    case 2: return launch_variant<false, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
-    case 4: return launch_variant<false, 2>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st);
+    case 1: return launch_variant<true, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
+    case 2: return launch_variant<false, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
+    case 4: return launch_variant<false, 2>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -737,6 +784,10 @@ void tc_shutdown() { host_cache_clear(); }
 extern "C" __attribute__((visibility("default"))) int mlra_trace_read(unsigned long long* host, size_t n) {
   const size_t bytes = sizeof(g_trace) < n * sizeof(unsigned long long) ? sizeof(g_trace) : n * sizeof(unsigned long long);
   return (int)cudaMemcpyFromSymbol(host, g_trace, bytes);
+}
+extern "C" __attribute__((visibility("default"))) int mlra_span_read(unsigned long long* host, size_t n) {
+  const size_t bytes = sizeof(g_span) < n * sizeof(unsigned long long) ? sizeof(g_span) : n * sizeof(unsigned long long);
+  return (int)cudaMemcpyFromSymbol(host, g_span, bytes);
 }
 #endif
 

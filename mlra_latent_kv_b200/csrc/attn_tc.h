@@ -15,9 +15,11 @@ bool tc_supported(int dtype, int H, int d_c, int d_r, int n_branch, int d_h, int
 
 // Launch the tcgen05 split-KV attention: same partial-result contract as the
 // CUDA-core kernel (slot c + b per worker piece, m/l per branch in log2 units).
+// pdl: launch as a programmatic dependent of the previous kernel in the stream
+// (its prologue overlaps that kernel; the queries are read after it completes).
 cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop, const int* page_table,
                              const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
-                             cudaStream_t st);
+                             cudaStream_t st, bool pdl);
 
 // Frees the host-side tensor-map cache.
 void tc_shutdown();

@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(128, 1)
   const int h = blockIdx.x, m0 = blockIdx.y * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = tmem_cols_for(a.Bp);
+  grid_dep_launch();  // the attention kernel may set up as this grid retires
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&full_bar), 1);
     mbar_init(smem_u32(&done_bar), 1);
@@ -98,18 +99,36 @@ __global__ void __launch_bounds__(128, 1)
       mma_commit(smem_u32(&done_bar));
     }
   }
-  // RoPE of the query (independent of the MMA)
-  if (blockIdx.y == 0) {
+  // RoPE of the query (independent of the MMA), spread over the head's
+  // d_c/128 blocks; the loads of a thread's pairs are issued before any use
+  {
     const int pairs = a.d_r / 2;
-    for (int idx = threadIdx.x; idx < a.B * pairs; idx += blockDim.x) {
-      const int b = idx / pairs, i = idx % pairs;
-      const __nv_bfloat16* src = q_rope + ((size_t)b * a.H + h) * a.d_r + 2 * i;
-      const float x0 = __bfloat162float(src[0]), x1 = __bfloat162float(src[1]);
-      float s, c;
-      rope_sincos(tab, i, __ldg(q_pos + b), &s, &c);
-      __nv_bfloat16* dst = q_ws + ((size_t)b * a.H + h) * (a.d_c + a.d_r) + a.d_c + 2 * i;
-      dst[0] = __float2bfloat16_rn((x0 * c - x1 * s) * a.q_scale);
-      dst[1] = __float2bfloat16_rn((x0 * s + x1 * c) * a.q_scale);
+    const int n = a.B * pairs, stride = blockDim.x * gridDim.y;
+    constexpr int kU = 4;
+    for (int base = blockIdx.y * blockDim.x + threadIdx.x; base < n; base += kU * stride) {
+      __nv_bfloat162 x[kU];
+      int pos[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int idx = base + u * stride;
+        if (idx < n) {
+          const int b = idx / pairs, i = idx % pairs;
+          x[u] = *reinterpret_cast<const __nv_bfloat162*>(q_rope + ((size_t)b * a.H + h) * a.d_r + 2 * i);
+          pos[u] = __ldg(q_pos + b);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int idx = base + u * stride;
+        if (idx < n) {
+          const int b = idx / pairs, i = idx % pairs;
+          const float x0 = __low2float(x[u]), x1 = __high2float(x[u]);
+          float sn, cs;
+          rope_sincos(tab, i, pos[u], &sn, &cs);
+          *reinterpret_cast<__nv_bfloat162*>(q_ws + ((size_t)b * a.H + h) * (a.d_c + a.d_r) + a.d_c + 2 * i) =
+              __floats2bfloat162_rn((x0 * cs - x1 * sn) * a.q_scale, (x0 * sn + x1 * cs) * a.q_scale);
+        }
+      }
     }
   }
   if (mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 21)) {
@@ -141,7 +160,8 @@ __global__ void __launch_bounds__(128, 1)
 //       o_lat[b, h, br cols] = branch_scale * sum_s 2^(m_s - M) o_s / L
 //   D (TMEM, 128 lanes x Bp)        -> out[b][h][m0 + lane] (bf16)
 // ---------------------------------------------------------------------------
-constexpr int kCuThreads = 256;
+constexpr int kCuThreads = 512;
+constexpr int kPieceUnroll = 4;  // partials of a row fetched together
 
 __global__ void __launch_bounds__(kCuThreads, 1)
     combine_upproj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ o_part,
@@ -150,10 +170,13 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int a_bytes = 2 * a.K * 128;             // K = d_c rows, two 64-column M blocks
-  uint8_t* sA = smem;
+  const int n_ml = (a.G + a.B - 1) * a.n_branch;  // (slot, branch) pairs
   uint8_t* sB = smem + a_bytes;                  // d_c/64 blocks of Bp rows
-  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * a.Bp * 128);  // [slots][n_branch]
-  int* s_c0 = reinterpret_cast<int*>(s_wt + (size_t)(a.G + a.B) * a.n_branch);
+  uint8_t* sA = smem;
+  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * a.Bp * 128);  // [slot][n_branch] piece weights
+  float* s_m = s_wt + n_ml;                                              // [slot][n_branch] running max
+  float* s_l = s_m + n_ml;                                               // [slot][n_branch] sum
+  int* s_c0 = reinterpret_cast<int*>(s_l + n_ml);
   int* s_c1 = s_c0 + a.B;
   __shared__ uint64_t full_bar, done_bar;
   __shared__ uint32_t tmem_base;
@@ -185,8 +208,8 @@ __global__ void __launch_bounds__(kCuThreads, 1)
       for (int r = 0; r < a.K; r += box_rows)
         tma_load_2d(smem_u32(sA + mb * a.K * 128 + r * 128), &tm_w, fb, m0 + 64 * mb, h * a.K + r);
   }
-  // sequence -> worker range (the split plan of the attention kernel)
-  if (warp == 0) {
+  if (warp == 1) {
+    // sequence -> worker range (the split plan of the attention kernel)
     long long T = 0;
     for (int base = 0; base < a.B; base += 32) {
       const int np = base + lane < a.B ? npages_of(seq_len_at(seq_lens, base + lane, maxL)) : 0;
@@ -205,32 +228,42 @@ __global__ void __launch_bounds__(kCuThreads, 1)
       prefix += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) s_T = T;
+    grid_dep_wait();
+  } else {
+    grid_dep_wait();  // the partials come from the attention kernel
+    // (m, l) of every slot of this head, all loads in flight at once
+    const int t = threadIdx.x - (threadIdx.x >= 64 ? 32 : 0), nt = blockDim.x - 32;
+    for (int i = t; i < n_ml; i += nt) {
+      const size_t base = (size_t)i * 2;
+      s_m[i] = ml_part[(base + 0) * a.H + h];
+      s_l[i] = ml_part[(base + 1) * a.H + h];
+    }
   }
   __syncthreads();
   const long long T = s_T;
-  // per (b, branch): weights of the pieces
+  // per (b, branch): weight of each piece, 2^(m_s - M) * branch_scale / L
   for (int idx = threadIdx.x; idx < a.B * a.n_branch; idx += blockDim.x) {
     const int b = idx / a.n_branch, br = idx % a.n_branch;
     const int c0 = s_c0[b], c1 = s_c1[b];
     float M = -INFINITY;
     for (int c = c0; c <= c1; ++c)
-      if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G))
-        M = fmaxf(M, ml_part[(((size_t)(c + b) * a.n_branch + br) * 2 + 0) * a.H + h]);
+      if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G)) M = fmaxf(M, s_m[(c + b) * a.n_branch + br]);
     float Lsum = 0.f;
     for (int c = c0; c <= c1; ++c)
       if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G)) {
-        const size_t base = ((size_t)(c + b) * a.n_branch + br) * 2;
-        Lsum += exp2f(ml_part[(base + 0) * a.H + h] - M) * ml_part[(base + 1) * a.H + h];
+        const int k = (c + b) * a.n_branch + br;
+        Lsum += exp2f(s_m[k] - M) * s_l[k];
       }
     const float scale = a.branch_scale / Lsum;
     for (int c = c0; c <= c1; ++c) {
       const bool nonempty = worker_start(c, T, a.G) != worker_start(c + 1, T, a.G);
-      s_wt[(size_t)(c + b) * a.n_branch + br] =
-          nonempty ? exp2f(ml_part[(((size_t)(c + b) * a.n_branch + br) * 2 + 0) * a.H + h] - M) * scale : 0.f;
+      const int k = (c + b) * a.n_branch + br;
+      s_wt[k] = nonempty ? exp2f(s_m[k] - M) * scale : 0.f;
     }
   }
   __syncthreads();
-  // o_lat rows (bf16) straight into the swizzled B operand; padding rows are zero
+  // o_lat rows (bf16) straight into the swizzled B operand; padding rows are
+  // zero.  The partials of up to kPieceUnroll pieces are fetched together.
   const int chunks = a.K / 8;
   const int d_cb = a.K / a.n_branch;
   for (int idx = threadIdx.x; idx < a.Bp * chunks; idx += blockDim.x) {
@@ -240,19 +273,33 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
     if (b < a.B) {
       const int br = (ch * 8) / d_cb;
-      for (int c = s_c0[b]; c <= s_c1[b]; ++c) {
-        const float w = s_wt[(size_t)(c + b) * a.n_branch + br];
-        if (w == 0.f) continue;
-        const float4* src = reinterpret_cast<const float4*>(o_part + (((size_t)(c + b) * chunks + ch) * a.H + h) * 8);
-        const float4 u = src[0], v = src[1];
-        acc[0] = fmaf(w, u.x, acc[0]);
-        acc[1] = fmaf(w, u.y, acc[1]);
-        acc[2] = fmaf(w, u.z, acc[2]);
-        acc[3] = fmaf(w, u.w, acc[3]);
-        acc[4] = fmaf(w, v.x, acc[4]);
-        acc[5] = fmaf(w, v.y, acc[5]);
-        acc[6] = fmaf(w, v.z, acc[6]);
-        acc[7] = fmaf(w, v.w, acc[7]);
+      const int c1 = s_c1[b];
+      for (int c = s_c0[b]; c <= c1; c += kPieceUnroll) {
+        float4 u[kPieceUnroll], v[kPieceUnroll];
+        float w[kPieceUnroll];
+#pragma unroll
+        for (int k = 0; k < kPieceUnroll; ++k) {
+          w[k] = c + k <= c1 ? s_wt[(c + k + b) * a.n_branch + br] : 0.f;
+          if (w[k] != 0.f) {
+            const float4* src =
+                reinterpret_cast<const float4*>(o_part + (((size_t)(c + k + b) * chunks + ch) * a.H + h) * 8);
+            u[k] = src[0];
+            v[k] = src[1];
+          } else {
+            u[k] = v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kPieceUnroll; ++k) {
+          acc[0] = fmaf(w[k], u[k].x, acc[0]);
+          acc[1] = fmaf(w[k], u[k].y, acc[1]);
+          acc[2] = fmaf(w[k], u[k].z, acc[2]);
+          acc[3] = fmaf(w[k], u[k].w, acc[3]);
+          acc[4] = fmaf(w[k], v[k].x, acc[4]);
+          acc[5] = fmaf(w[k], v[k].y, acc[5]);
+          acc[6] = fmaf(w[k], v[k].z, acc[6]);
+          acc[7] = fmaf(w[k], v[k].w, acc[7]);
+        }
       }
     }
     uint4 pk;
@@ -309,13 +356,19 @@ bool absorb_tc_supported(int dtype, int B, int d_h, int d_c) {
   return dtype == 1 && B >= 1 && B <= 256 && d_h % 64 == 0 && d_h <= 256 && d_c % 128 == 0;
 }
 
-// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B) plus d_c/64 x Bp x 128 B of o_lat rows
-bool upproj_tc_supported(int dtype, int B, int d_c, int d_v) {
-  return dtype == 1 && B >= 1 && B <= 96 && d_c % 64 == 0 && d_c <= 512 && (d_c <= 256 || d_c % 256 == 0) &&
-         d_v % 128 == 0;
+int batch_pad(int B) { return B <= 16 ? 16 : (B + 15) / 16 * 16; }
+
+// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B), d_c/64 x Bp x 128 B
+// of o_lat rows, the (m, l, weight) of every slot and branch, two ints per row
+static size_t upproj_smem_bytes(int B, int d_c, int G, int n_branch) {
+  return 1024 + (size_t)2 * d_c * 128 + (size_t)(d_c / 64) * batch_pad(B) * 128 +
+         (size_t)3 * (G + B) * n_branch * 4 + (size_t)2 * B * 4;
 }
 
-int batch_pad(int B) { return B <= 16 ? 16 : (B + 15) / 16 * 16; }
+bool upproj_tc_supported(int dtype, int B, int d_c, int d_v, int G, int n_branch) {
+  return dtype == 1 && B >= 1 && B <= 96 && d_c % 64 == 0 && d_c <= 512 && (d_c <= 256 || d_c % 256 == 0) &&
+         d_v % 128 == 0 && upproj_smem_bytes(B, d_c, G, n_branch) <= 232448;
+}
 
 cudaError_t launch_absorb_tc(const void* q_nope, const void* q_rope, const int* q_pos, const void* W_UK, void* q_ws,
                              int* err, const GemmArgs& a, const RopeTable& tab, cudaStream_t st) {
@@ -332,16 +385,25 @@ cudaError_t launch_absorb_tc(const void* q_nope, const void* q_rope, const int* 
 }
 
 cudaError_t launch_combine_upproj_tc(const float* o_part, const float* ml_part, const int* seq_lens, const void* W_UV,
-                                     void* out, int* err, const GemmArgs& a, cudaStream_t st) {
+                                     void* out, int* err, const GemmArgs& a, cudaStream_t st, bool pdl) {
   CUtensorMap tw;
   if (!tmap_2d(&tw, W_UV, (uint64_t)a.N_out, (uint64_t)a.H * a.K, 64, (uint32_t)(a.K < 256 ? a.K : 256)))
     return cudaErrorInvalidValue;
-  const int smem = 1024 + 2 * a.K * 128 + (a.K / 64) * a.Bp * 128 + (a.G + a.B) * a.n_branch * 4 + 2 * a.B * 4;
+  const int smem = (int)upproj_smem_bytes(a.B, a.K, a.G, a.n_branch);
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(combine_upproj_tc_kernel), smem);
   if (e != cudaSuccess) return e;
-  combine_upproj_tc_kernel<<<dim3(a.H, a.N_out / 128), kCuThreads, smem, st>>>(
-      tw, o_part, ml_part, seq_lens, (__nv_bfloat16*)out, err, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.H, a.N_out / 128, 1);
+  cfg.blockDim = dim3(kCuThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, combine_upproj_tc_kernel, tw, o_part, ml_part, seq_lens, (__nv_bfloat16*)out, err,
+                            a);
 }
 
 }  // namespace mlra

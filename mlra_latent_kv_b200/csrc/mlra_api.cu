@@ -163,7 +163,7 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
   cudaError_t e;
 
   const bool tc_absorb = p.tc && absorb_tc_supported(d->dtype, d->B, d->d_h, d->d_c);
-  const bool tc_upproj = p.tc && upproj_tc_supported(d->dtype, d->B, d->d_c, d->d_v);
+  const bool tc_upproj = p.tc && upproj_tc_supported(d->dtype, d->B, d->d_c, d->d_v, p.G, d->n_branch);
   // The tcgen05 attention kernel takes queries pre-multiplied by scale*log2(e)
   // (its scores are then base-2 logits directly); the CUDA-core kernel scales itself.
   const float scale_log2 = scale_of(d) * 1.4426950408889634f;
@@ -184,7 +184,12 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
   AttnArgs at{d->B, d->H, d->d_c, d->d_r, d->n_branch, d->max_pages_per_seq, d->num_pages, p.G,
               p.tc ? 1.0f : scale_log2};
   if (p.tc) {
-    e = launch_attend_tc(q_ws, latent_cache, rope_cache, page_table, seq_lens, o_part, ml_part, err, at, stream);
+    // Programmatic dependent launches chain absorption -> attention -> combine
+    // (not when stage events sit between the kernels).  The absorption kernel
+    // itself is an ordinary launch, so every earlier kernel of the stream (the
+    // cache append) has completed before any of the three starts.
+    e = launch_attend_tc(q_ws, latent_cache, rope_cache, page_table, seq_lens, o_part, ml_part, err, at, stream,
+                         tc_absorb && ev == nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 attention launch");
   } else {
     e = launch_attend_simt(d->dtype, static_cast<const float*>(q_ws), latent_cache, rope_cache, page_table, seq_lens,
@@ -197,7 +202,7 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
     if (ev) record_event(ev[3], stream);
     GemmArgs gu = ga;
     gu.K = d->d_c;
-    e = launch_combine_upproj_tc(o_part, ml_part, seq_lens, W_UV, out, err, gu, stream);
+    e = launch_combine_upproj_tc(o_part, ml_part, seq_lens, W_UV, out, err, gu, stream, ev == nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "combine + up-projection launch");
   } else {
     CombineArgs ca{d->B, d->H, d->d_c, d->n_branch, p.G, d->max_pages_per_seq, branch_scale};

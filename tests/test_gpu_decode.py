@@ -130,10 +130,11 @@ def test_dominant_key_is_selected(kernel):
     assert err <= tol
 
 
-def test_device_check_bad_page_id():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_device_check_bad_page_id(kernel):
     w = synth.workload("dsv2_contiguous").with_(B=2, seq_len=100)
     inp = synth.make_inputs(w)
-    s = DecodeSession(w, inp, kernel="simt")
+    s = DecodeSession(w, inp, kernel=kernel)
     s.page_table[1, 1] = 10_000_000  # outside the pool
     s.decode()
     with pytest.raises(abi.MlraError) as ei:
@@ -158,3 +159,28 @@ def test_full_size_sampled(name):
     err, tol, out, ref, _ = run_case(w, "auto", pairs=FULL_PAIRS[name])
     assert err <= tol, f"{name}: {err:.3e} > {tol:.3e}"
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("name", ["dsv2_contiguous", "mlra4"])
+def test_staged_and_graph_launches_bitwise(name):
+    """The launch with stage events between the kernels (serialised), an eager
+    plain launch and a CUDA-graph replay of the plain launch (kernels chained by
+    programmatic dependent launch) give the same output bits."""
+    w = synth.workload(name).with_(B=4, seq_len=1000)
+    s = DecodeSession(w, synth.make_inputs(w))
+    o1 = s.step().clone()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for e in ev:
+        e.record()
+    o2 = s.step(events=ev).clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        s.step()
+    s.out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    o3 = s.out.clone()
+    s.check()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
+    assert ev[1].elapsed_time(ev[2]) > 0
