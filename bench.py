@@ -115,10 +115,15 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": sorted(self.reasons)}
 
 
+ATTN_SOURCES = ("attn_tc.cu", "attn_tc.h", "ptx.cuh", "common.cuh", "launch.h", "host_cache.cu", "host_cache.h")
+
+
 def source_digest() -> str:
+    """Digest of the sources the attention kernel is built from (a stored ncu
+    traffic figure is used only while it matches)."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "mlra_latent_kv_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "mlra_latent_kv_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
