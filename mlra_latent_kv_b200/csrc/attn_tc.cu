@@ -491,7 +491,6 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
         if (progressed) {
           t_idle = 0;
         } else {
-          __nanosleep(32);  // idle: leave issue slots to the softmax warp sharing this sub-partition
           if (*abort_flag) {
             ok = false;
             break;
@@ -687,7 +686,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int d = d0 + 8 * q;
-              float4* dst = reinterpret_cast<float4*>(o_part + (((size_t)slot * (a.d_c / 8) + d / 8) * a.H + row) * 8);
+              float4* dst = reinterpret_cast<float4*>(o_part + ((size_t)slot * a.H + row) * a.d_c + d);
               dst[0] = make_float4(__uint_as_float(o[8 * q]), __uint_as_float(o[8 * q + 1]),
                                    __uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
               dst[1] = make_float4(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]),

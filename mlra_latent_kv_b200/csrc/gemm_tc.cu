@@ -28,6 +28,21 @@ namespace {
 
 using namespace ptx;
 
+// Optional phase trace (builds with -DMLRA_TRACE only): globaltimer stamps of
+// each CTA's phases, [kernel][cta][event].
+#ifdef MLRA_TRACE
+__device__ unsigned long long g_gtrace[2][1024][8];
+#define GEMM_TRACE(k, ev)                                                                      \
+  do {                                                                                         \
+    const int cta_ = blockIdx.x * gridDim.y + blockIdx.y;                                      \
+    if (threadIdx.x == 0 && cta_ < 1024) g_gtrace[k][cta_][ev] = globaltimer_ns();              \
+  } while (0)
+#else
+#define GEMM_TRACE(k, ev) \
+  do {                    \
+  } while (0)
+#endif
+
 // 128-byte-swizzled K-major tile of `rows` rows x 64 bf16: byte offset of the
 // 16-byte chunk (row, chunk) -- the layout TMA writes and the MMA reads.
 __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
@@ -63,6 +78,7 @@ __global__ void __launch_bounds__(128, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = tmem_cols_for(a.Bp);
   grid_dep_launch();  // the attention kernel may set up as this grid retires
+  GEMM_TRACE(0, 0);
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&full_bar), 1);
     mbar_init(smem_u32(&done_bar), 1);
@@ -77,27 +93,11 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  bool ok = true;
-  if (threadIdx.x == 0) {
-    const uint32_t fb = smem_u32(&full_bar);
+  const uint32_t fb = smem_u32(&full_bar);
+  if (threadIdx.x == 0) {  // weights and queries in flight while the RoPE below runs
     mbar_expect_tx(fb, a_bytes + (a.K / 64) * a.Bp * 128);
     for (int mb = 0; mb < 2; ++mb) tma_load_2d(smem_u32(sA + mb * a.K * 128), &tm_w, fb, m0 + 64 * mb, h * a.K);
     for (int kb = 0; kb < a.K / 64; ++kb) tma_load_3d(smem_u32(sB + kb * a.Bp * 128), &tm_q, fb, 64 * kb, h, 0);
-    ok = mbar_wait(fb, 0, &abort_flag, err, 20);
-    if (ok) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, a.Bp, true, false);
-      const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
-      const uint64_t bd0 = sdesc_sw128(smem_u32(sB), 16, 1024);
-      const uint64_t bkb = (uint64_t)((a.Bp * 128) >> 4);
-      for (int kb = 0; kb < a.K / 64; ++kb) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_ss(tmem, ad0 + (uint64_t)(kb * 4 + ks) * 128u, bd0 + kb * bkb + (uint64_t)(ks * 2), idesc,
-                 (kb | ks) ? 1u : 0u);
-      }
-      mma_commit(smem_u32(&done_bar));
-    }
   }
   // RoPE of the query (independent of the MMA), spread over the head's
   // d_c/128 blocks; the loads of a thread's pairs are issued before any use
@@ -131,7 +131,24 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   }
+  if (threadIdx.x == 0 && mbar_wait(fb, 0, &abort_flag, err, 20)) {
+    GEMM_TRACE(0, 2);
+    tc_fence_after();
+    const uint32_t idesc = idesc_bf16_f32(128, a.Bp, true, false);
+    const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
+    const uint64_t bd0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+    const uint64_t bkb = (uint64_t)((a.Bp * 128) >> 4);
+    for (int kb = 0; kb < a.K / 64; ++kb) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_ss(tmem, ad0 + (uint64_t)(kb * 4 + ks) * 128u, bd0 + kb * bkb + (uint64_t)(ks * 2), idesc,
+               (kb | ks) ? 1u : 0u);
+    }
+    mma_commit(smem_u32(&done_bar));
+  }
+  GEMM_TRACE(0, 3);
   if (mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 21)) {
+    GEMM_TRACE(0, 4);
     tc_fence_after();
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     for (int cc = 0; cc < a.Bp; cc += 32) {
@@ -150,6 +167,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, ncols);
+  GEMM_TRACE(0, 5);
 }
 
 // ---------------------------------------------------------------------------
@@ -178,6 +196,7 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   float* s_l = s_m + n_ml;                                               // [slot][n_branch] sum
   int* s_c0 = reinterpret_cast<int*>(s_l + n_ml);
   int* s_c1 = s_c0 + a.B;
+  int* s_ne = s_c1 + a.B;  // [G] worker has pages
   __shared__ uint64_t full_bar, done_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
@@ -186,6 +205,7 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ncols = tmem_cols_for(a.Bp);
   const int maxL = a.maxp * kPage;
+  GEMM_TRACE(1, 0);
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&full_bar), 1);
     mbar_init(smem_u32(&done_bar), 1);
@@ -228,91 +248,116 @@ __global__ void __launch_bounds__(kCuThreads, 1)
       prefix += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) s_T = T;
-    grid_dep_wait();
-  } else {
-    grid_dep_wait();  // the partials come from the attention kernel
-    // (m, l) of every slot of this head, all loads in flight at once
-    const int t = threadIdx.x - (threadIdx.x >= 64 ? 32 : 0), nt = blockDim.x - 32;
-    for (int i = t; i < n_ml; i += nt) {
-      const size_t base = (size_t)i * 2;
-      s_m[i] = ml_part[(base + 0) * a.H + h];
-      s_l[i] = ml_part[(base + 1) * a.H + h];
-    }
   }
   __syncthreads();
-  const long long T = s_T;
+  {
+    // workers with an empty page range wrote no partial: flag them once
+    const long long T = s_T;
+    for (int c = threadIdx.x; c < a.G; c += blockDim.x)
+      s_ne[c] = worker_start(c, T, a.G) != worker_start(c + 1, T, a.G) ? 1 : 0;
+  }
+  grid_dep_wait();  // the partials come from the attention kernel
+  // (m, l) of every slot of this head, all loads in flight at once
+  for (int i = threadIdx.x; i < n_ml; i += blockDim.x) {
+    const size_t base = (size_t)i * 2;
+    s_m[i] = ml_part[(base + 0) * a.H + h];
+    s_l[i] = ml_part[(base + 1) * a.H + h];
+  }
+  __syncthreads();
+  GEMM_TRACE(1, 1);
   // per (b, branch): weight of each piece, 2^(m_s - M) * branch_scale / L
   for (int idx = threadIdx.x; idx < a.B * a.n_branch; idx += blockDim.x) {
     const int b = idx / a.n_branch, br = idx % a.n_branch;
     const int c0 = s_c0[b], c1 = s_c1[b];
     float M = -INFINITY;
     for (int c = c0; c <= c1; ++c)
-      if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G)) M = fmaxf(M, s_m[(c + b) * a.n_branch + br]);
+      if (s_ne[c]) M = fmaxf(M, s_m[(c + b) * a.n_branch + br]);
     float Lsum = 0.f;
     for (int c = c0; c <= c1; ++c)
-      if (worker_start(c, T, a.G) != worker_start(c + 1, T, a.G)) {
+      if (s_ne[c]) {
         const int k = (c + b) * a.n_branch + br;
         Lsum += exp2f(s_m[k] - M) * s_l[k];
       }
     const float scale = a.branch_scale / Lsum;
     for (int c = c0; c <= c1; ++c) {
-      const bool nonempty = worker_start(c, T, a.G) != worker_start(c + 1, T, a.G);
       const int k = (c + b) * a.n_branch + br;
-      s_wt[k] = nonempty ? exp2f(s_m[k] - M) * scale : 0.f;
+      s_wt[k] = s_ne[c] ? exp2f(s_m[k] - M) * scale : 0.f;
     }
   }
   __syncthreads();
+  GEMM_TRACE(1, 2);
   // o_lat rows (bf16) straight into the swizzled B operand; padding rows are
-  // zero.  The partials of up to kPieceUnroll pieces are fetched together.
+  // zero.  A thread takes two (row, 8-dim chunk) items at a time and fetches
+  // the partials of up to kPieceUnroll pieces of both before using any.
   const int chunks = a.K / 8;
   const int d_cb = a.K / a.n_branch;
-  for (int idx = threadIdx.x; idx < a.Bp * chunks; idx += blockDim.x) {
-    const int b = idx / chunks, ch = idx % chunks;
-    float acc[8];
+  const int n_items = a.Bp * chunks;
+  for (int base = threadIdx.x; base < n_items; base += 2 * blockDim.x) {
+    int bq[2], chq[2], c0q[2], c1q[2], brq[2];
+    float acc[2][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    if (b < a.B) {
-      const int br = (ch * 8) / d_cb;
-      const int c1 = s_c1[b];
-      for (int c = s_c0[b]; c <= c1; c += kPieceUnroll) {
-        float4 u[kPieceUnroll], v[kPieceUnroll];
-        float w[kPieceUnroll];
+    for (int u = 0; u < 2; ++u) {
+      const int idx = base + u * blockDim.x;
+      bq[u] = idx < n_items ? idx / chunks : a.Bp;
+      chq[u] = idx % chunks;
+      const bool row = bq[u] < a.B;
+      c0q[u] = row ? s_c0[bq[u]] : 0;
+      c1q[u] = row ? s_c1[bq[u]] : -1;
+      brq[u] = (chq[u] * 8) / d_cb;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[u][j] = 0.f;
+    }
+    const int np = max(c1q[0] - c0q[0], c1q[1] - c0q[1]) + 1;
+    for (int k0 = 0; k0 < np; k0 += kPieceUnroll) {
+      float4 uv[2][kPieceUnroll][2];
+      float w[2][kPieceUnroll];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
         for (int k = 0; k < kPieceUnroll; ++k) {
-          w[k] = c + k <= c1 ? s_wt[(c + k + b) * a.n_branch + br] : 0.f;
-          if (w[k] != 0.f) {
+          const int c = c0q[u] + k0 + k;
+          w[u][k] = c <= c1q[u] ? s_wt[(c + bq[u]) * a.n_branch + brq[u]] : 0.f;
+          if (w[u][k] != 0.f) {
             const float4* src =
-                reinterpret_cast<const float4*>(o_part + (((size_t)(c + k + b) * chunks + ch) * a.H + h) * 8);
-            u[k] = src[0];
-            v[k] = src[1];
+                reinterpret_cast<const float4*>(o_part + ((size_t)(c + bq[u]) * a.H + h) * a.K + chq[u] * 8);
+            uv[u][k][0] = src[0];
+            uv[u][k][1] = src[1];
           } else {
-            u[k] = v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            uv[u][k][0] = uv[u][k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
 #pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
         for (int k = 0; k < kPieceUnroll; ++k) {
-          acc[0] = fmaf(w[k], u[k].x, acc[0]);
-          acc[1] = fmaf(w[k], u[k].y, acc[1]);
-          acc[2] = fmaf(w[k], u[k].z, acc[2]);
-          acc[3] = fmaf(w[k], u[k].w, acc[3]);
-          acc[4] = fmaf(w[k], v[k].x, acc[4]);
-          acc[5] = fmaf(w[k], v[k].y, acc[5]);
-          acc[6] = fmaf(w[k], v[k].z, acc[6]);
-          acc[7] = fmaf(w[k], v[k].w, acc[7]);
+          const float wk = w[u][k];
+          acc[u][0] = fmaf(wk, uv[u][k][0].x, acc[u][0]);
+          acc[u][1] = fmaf(wk, uv[u][k][0].y, acc[u][1]);
+          acc[u][2] = fmaf(wk, uv[u][k][0].z, acc[u][2]);
+          acc[u][3] = fmaf(wk, uv[u][k][0].w, acc[u][3]);
+          acc[u][4] = fmaf(wk, uv[u][k][1].x, acc[u][4]);
+          acc[u][5] = fmaf(wk, uv[u][k][1].y, acc[u][5]);
+          acc[u][6] = fmaf(wk, uv[u][k][1].z, acc[u][6]);
+          acc[u][7] = fmaf(wk, uv[u][k][1].w, acc[u][7]);
         }
-      }
     }
-    uint4 pk;
-    pk.x = pack_bf16x2(acc[0], acc[1]);
-    pk.y = pack_bf16x2(acc[2], acc[3]);
-    pk.z = pack_bf16x2(acc[4], acc[5]);
-    pk.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(sB + (ch / 8) * a.Bp * 128 + sw128_off(b, ch % 8)) = pk;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (bq[u] >= a.Bp) continue;
+      uint4 pk;
+      pk.x = pack_bf16x2(acc[u][0], acc[u][1]);
+      pk.y = pack_bf16x2(acc[u][2], acc[u][3]);
+      pk.z = pack_bf16x2(acc[u][4], acc[u][5]);
+      pk.w = pack_bf16x2(acc[u][6], acc[u][7]);
+      *reinterpret_cast<uint4*>(sB + (chq[u] / 8) * a.Bp * 128 + sw128_off(bq[u], chq[u] % 8)) = pk;
+    }
   }
   fence_proxy_async_smem();
   __syncthreads();
+  GEMM_TRACE(1, 3);
   if (threadIdx.x == 0) {
     if (mbar_wait(smem_u32(&full_bar), 0, &abort_flag, err, 22)) {
+      GEMM_TRACE(1, 4);
       tc_fence_after();
       const uint32_t idesc = idesc_bf16_f32(128, a.Bp, true, false);
       const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
@@ -328,6 +373,7 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     }
   }
   if (warp < 4 && mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 23)) {
+    GEMM_TRACE(1, 5);
     tc_fence_after();
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     for (int cc = 0; cc < a.Bp; cc += 32) {
@@ -345,6 +391,7 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, ncols);
+  GEMM_TRACE(1, 6);
 }
 
 // ---------------------------------------------------------------------------
@@ -359,10 +406,11 @@ bool absorb_tc_supported(int dtype, int B, int d_h, int d_c) {
 int batch_pad(int B) { return B <= 16 ? 16 : (B + 15) / 16 * 16; }
 
 // shared memory: the whole W_UV[h] slice (2 x d_c x 128 B), d_c/64 x Bp x 128 B
-// of o_lat rows, the (m, l, weight) of every slot and branch, two ints per row
+// of o_lat rows, the (m, l, weight) of every slot and branch, two ints per row,
+// one flag per worker
 static size_t upproj_smem_bytes(int B, int d_c, int G, int n_branch) {
   return 1024 + (size_t)2 * d_c * 128 + (size_t)(d_c / 64) * batch_pad(B) * 128 +
-         (size_t)3 * (G + B) * n_branch * 4 + (size_t)2 * B * 4;
+         (size_t)3 * (G + B) * n_branch * 4 + (size_t)2 * B * 4 + (size_t)G * 4;
 }
 
 bool upproj_tc_supported(int dtype, int B, int d_c, int d_v, int G, int n_branch) {
@@ -405,5 +453,14 @@ cudaError_t launch_combine_upproj_tc(const float* o_part, const float* ml_part, 
   return cudaLaunchKernelEx(&cfg, combine_upproj_tc_kernel, tw, o_part, ml_part, seq_lens, (__nv_bfloat16*)out, err,
                             a);
 }
+
+#ifdef MLRA_TRACE
+// Copies the phase trace of the last absorption / combine launches (trace builds only).
+extern "C" __attribute__((visibility("default"))) int mlra_gemm_trace_read(unsigned long long* host, size_t n) {
+  const size_t bytes =
+      sizeof(g_gtrace) < n * sizeof(unsigned long long) ? sizeof(g_gtrace) : n * sizeof(unsigned long long);
+  return (int)cudaMemcpyFromSymbol(host, g_gtrace, bytes);
+}
+#endif
 
 }  // namespace mlra

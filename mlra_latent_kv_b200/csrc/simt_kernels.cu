@@ -80,9 +80,8 @@ __global__ void __launch_bounds__(128) absorb_kernel(const T* __restrict__ q_nop
 // Lane l owns latent dims l + 32k and rope dims l + 32k.
 // Writes the unnormalised partial o (relative to the running max m, in log2
 // units) and m, l per branch to slot c + b.  Partial layout (shared with the
-// tcgen05 kernels): o_part[slot][d_c/8][H][8] fp32 (32-byte chunks, so a head
-// per thread writes and a head per block reads whole sectors),
-// ml_part[slot][n_branch][2][H] (m, l).
+// tcgen05 kernels): o_part[slot][H][d_c] fp32 (head-major, so the combine of a
+// head reads each piece's row contiguously), ml_part[slot][n_branch][2][H] (m, l).
 // ---------------------------------------------------------------------------
 constexpr int kTileTok = 16;
 constexpr int kMaxDpl = 16;  // d_c <= 512
@@ -183,7 +182,7 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(const float* __restric
       for (int k = 0; k < kMaxDpl; ++k) {
         if (k < dpl) {
           const int d = lane + 32 * k;
-          o_part[(((size_t)slot * (a.d_c / 8) + d / 8) * a.H + h) * 8 + (d & 7)] = o[k];
+          o_part[((size_t)slot * a.H + h) * a.d_c + d] = o[k];
         }
       }
       if (lane == 0) {
@@ -253,7 +252,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
         if (MLRA_WORKER_EMPTY(c)) continue;
         const size_t base = ((size_t)(c + b) * a.n_branch + br) * 2;
         const float w = exp2f(ml_part[(base + 0) * a.H + h] - M);
-        acc = fmaf(w, o_part[(((size_t)(c + b) * (a.d_c / 8) + d / 8) * a.H + h) * 8 + (d & 7)], acc);
+        acc = fmaf(w, o_part[((size_t)(c + b) * a.H + h) * a.d_c + d], acc);
       }
       dst[d] = from_f<OT>(acc * inv);
     }

@@ -114,6 +114,6 @@ class DecodeSession:
               and w.n_branch in (1, 2, 4))
         G = self.dims.num_splits or torch.cuda.get_device_properties(self.device).multi_processor_count // 2
         bp = 16 if w.B <= 16 else (w.B + 15) // 16 * 16
-        smem = 1024 + 2 * w.d_c * 128 + (w.d_c // 64) * bp * 128 + 3 * (G + w.B) * w.n_branch * 4 + 2 * w.B * 4
+        smem = 1024 + 2 * w.d_c * 128 + (w.d_c // 64) * bp * 128 + 3 * (G + w.B) * w.n_branch * 4 + 2 * w.B * 4 + G * 4
         fused = tc and w.B <= 96 and w.d_v % 128 == 0 and smem <= 232448
         return (2 if self.appends else 0) + 2 + (1 if fused else 2)
