@@ -173,10 +173,14 @@ def pick_pairs(w, n, seed=0):
 
 def cpu_baseline(w, inp, budget_s: float = 15.0) -> dict:
     """The oracle (as it stands) on a bounded sample of (b, h) pairs, scaled to a full step."""
-    t8 = time_oracle_pairs(w, inp, pick_pairs(w, 8, seed=7)) / 8
-    n = max(1, min(w.B * w.H, int(budget_s / max(t8, 1e-6))))
-    pairs = pick_pairs(w, n, seed=1)
-    t = time_oracle_pairs(w, inp, pairs)
+    time_oracle_pairs(w, inp, pick_pairs(w, 8, seed=6))  # warm (first-touch costs are not the oracle's rate)
+    # grow the sample until it takes about half the budget or covers the whole step (the
+    # oracle's per-pair cost falls with the sample size, so one small calibration overshoots)
+    n = min(w.B * w.H, 64)
+    t = time_oracle_pairs(w, inp, pick_pairs(w, n, seed=1))
+    while t < 0.5 * budget_s and n < w.B * w.H:
+        n = min(w.B * w.H, max(n + 1, int(n * budget_s / max(t, 1e-3))))
+        t = time_oracle_pairs(w, inp, pick_pairs(w, n, seed=1))
     per_pair = t / n
     step_s = per_pair * w.B * w.H
     sb = step_bytes(w, inp)
