@@ -51,11 +51,9 @@ using namespace ptx;
 // warpgroup covers the 128 TMEM lanes = heads)
 template <bool kExch, int kBrPerCta>
 constexpr int threads_of() { return 64 + 128 * kBrPerCta + (kExch ? 128 : 0); }  // + MLA exchange warps
-constexpr int kQSlotBytes = 128 * 128;    // 128 query rows x 64 bf16
 constexpr int kTileSlotBytes = 64 * 128;  // 64 tokens x 64 bf16
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kXBytes = 64 * 128 * 2;     // one page of fp16 partial scores, 128 rows
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kIdAhead = 8;               // page ids read this many pages before their tile
 constexpr int kIdRing = 16;
@@ -86,22 +84,34 @@ struct Bars {
 //  buffer for the partial scores of one page.
 //  MLRA: 4 latent blocks + the full rope block (128-byte swizzle) per stage,
 //  ring of 3 stages.
-template <bool kExch>
+//  Query blocks, the exchange buffer and the rope query take kHq rows: 128,
+//  or 32 when H <= 32, which leaves room for two more stages.  The M = 128
+//  MMAs read 128 rows from each query block; the rows past kHq fall on the
+//  next buffer, feed only MMA rows of absent heads, and are never used.
+template <bool kExch, int kHq>
 struct Layout {
-  static constexpr int kStages = kExch ? 4 : 3;
-  static constexpr int kRopeQBytes = kExch ? 128 * 64 : kQSlotBytes;
+  static constexpr int kQSlotBytes = kHq * 128;  // kHq query rows x 64 bf16
+  static constexpr int kRopeQBytes = kExch ? kHq * 64 : kQSlotBytes;
   static constexpr int kRopeTileBytes = kExch ? 64 * 64 : kTileSlotBytes;
   static constexpr int kRopeRowBytes = kExch ? 64 : 128;
+  static constexpr int kXBytes = 64 * kHq * 2;   // one page of fp16 partial scores, kHq rows
   static constexpr int kStageBytes = 4 * kTileSlotBytes + (kExch ? 0 : kRopeTileBytes);
   static constexpr int kQ = 0;
   static constexpr int kQRope = 4 * kQSlotBytes;
-  static constexpr int kTile = kQRope + kRopeQBytes;
-  static constexpr int kRope = kTile + kStages * kStageBytes;  // MLA rope ring
+  static constexpr int kRope = kQRope + kRopeQBytes;  // MLA rope ring
   static constexpr int kX = kRope + (kExch ? 2 * kRopeTileBytes : 0);
-  static constexpr int kBars = kX + (kExch ? kXBytes : 0);
-  static constexpr int kBytes = kBars + (int)sizeof(Bars) + 1024;  // + alignment slack
-  static_assert(kStageBytes % 1024 == 0 && kTile % 1024 == 0 && kRope % 1024 == 0, "aligned slots");
+  static constexpr int kTile = (kX + (kExch ? kXBytes : 0) + 1023) / 1024 * 1024;
+  static constexpr int kFixed = kTile + (int)sizeof(Bars) + 1024;  // + alignment slack
+  static constexpr int kStages = (232448 - kFixed) / kStageBytes < kMaxStages ? (232448 - kFixed) / kStageBytes
+                                                                                : kMaxStages;
+  static constexpr int kBars = kTile + kStages * kStageBytes;
+  static constexpr int kBytes = kBars + (int)sizeof(Bars) + 1024;
+  static_assert(kStages >= 3, "stage ring");
+  static_assert(kStageBytes % 1024 == 0 && kTile % 1024 == 0 && kRope % 512 == 0 && kQRope % 1024 == 0,
+                "aligned slots");
   static_assert(kBytes <= 232448, "shared memory");
+  // the last query block's 128-row MMA read stays inside the CTA's shared memory
+  static_assert(3 * kQSlotBytes + 128 * 128 <= kBytes && kQRope + 128 * (kExch ? 64 : 128) <= kBytes, "query reads");
 };
 
 // Optional pipeline trace (builds with -DMLRA_TRACE only): globaltimer stamps
@@ -194,13 +204,14 @@ __device__ __forceinline__ bool softmax_page(float (&s)[64], int valid, bool fir
   return rescale;
 }
 
-template <bool kExch, int kBrPerCta>
+template <bool kExch, int kBrPerCta, int kHq>
 __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rope,
                      const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
                      const int* __restrict__ page_table, const int* __restrict__ seq_lens,
                      float* __restrict__ o_part, float* __restrict__ ml_part, int* __restrict__ err, AttnArgs a) {
-  using L = Layout<kExch>;
+  using L = Layout<kExch, kHq>;
+  constexpr int kQSlotBytes = L::kQSlotBytes;
   constexpr int kLatPerBr = 4 / kBrPerCta;      // latent slots per branch
   constexpr int kPvN = 256 / kBrPerCta;         // PV output columns per branch
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
@@ -555,7 +566,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
           if (real) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-              st_async_v4(dst + (uint32_t)((q * 128 + row) * 16), h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3],
+              st_async_v4(dst + (uint32_t)((q * kHq + row) * 16), h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3],
                           bar);
           }
           if (row == 0) MLRA_TRACE_EV(g, kEvSent);
@@ -607,7 +618,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
           if (real) {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              const uint4 v = *reinterpret_cast<const uint4*>(sX + (q * 128 + row) * 16);
+              const uint4 v = *reinterpret_cast<const uint4*>(sX + (q * kHq + row) * 16);
               const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
@@ -719,13 +730,13 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
 // ---------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
-template <bool kExch, int kBrPerCta>
+template <bool kExch, int kBrPerCta, int kHq>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tl, const CUtensorMap& tr,
                            const int* page_table,
                            const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                            cudaStream_t st, bool pdl) {
-  auto kern = attend_tc_kernel<kExch, kBrPerCta>;
-  const int smem = Layout<kExch>::kBytes;
+  auto kern = attend_tc_kernel<kExch, kBrPerCta, kHq>;
+  const int smem = Layout<kExch, kHq>::kBytes;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -768,12 +779,16 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
     tqr = tq;
     if (!tmap_2d(&tr, rop, (uint64_t)a.d_r, (uint64_t)a.num_pages * kPage, 64, 64)) return cudaErrorInvalidValue;
   }
+#define MLRA_LAUNCH(E, BR, HQ) \
+  launch_variant<E, BR, HQ>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl)
+  const bool small = a.H <= 32;  // compact query buffers, deeper ring
   switch (a.n_branch) {
-    case 1: return launch_variant<true, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
-    case 2: return launch_variant<false, 1>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
-    case 4: return launch_variant<false, 2>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
+    case 1: return small ? MLRA_LAUNCH(true, 1, 32) : MLRA_LAUNCH(true, 1, 128);
+    case 2: return small ? MLRA_LAUNCH(false, 1, 32) : MLRA_LAUNCH(false, 1, 128);
+    case 4: return small ? MLRA_LAUNCH(false, 2, 32) : MLRA_LAUNCH(false, 2, 128);
     default: return cudaErrorInvalidValue;
   }
+#undef MLRA_LAUNCH
 }
 
 void tc_shutdown() { host_cache_clear(); }
