@@ -14,24 +14,32 @@
 //   * A worker is a pair of CTAs (on two SMs).  The fp32 accumulator O of 128
 //     heads x 512 latent dims needs all 512 TMEM columns of an SM, so each CTA
 //     of the pair owns 256 latent dims of O (and loads only those 256 dims of
-//     every cache tile); TMEM then also holds a double-buffered S.
+//     every cache page); the other 256 TMEM columns hold a ring of S buffers
+//     (four with one branch per CTA, two with two).
 //   * MLA (one softmax over all 512 dims): CTA r computes the partial scores
-//     of its 256 dims (CTA 0 adds the rope part) and the two partials are
-//     exchanged through distributed shared memory, so both CTAs hold the same
-//     full S and compute bit-identical softmax weights.
+//     of its 256 latent dims and of its 32 of the 64 rope dims.  Exchange warps
+//     send each page's partial (rounded to fp16) to the peer through
+//     distributed shared memory as soon as QK^T has produced it; both CTAs add
+//     f16(own) + f16(peer's), so they hold the same bits and compute identical
+//     softmax weights.
 //   * MLRA with 2 or 4 branches: the branches of a CTA are wholly its own, so
 //     the pair never talks; each CTA adds the full rope score to its branches.
-//   * Per 64-token page: one TMA producer warp loads the page's latent dims
-//     and rope key (128-byte swizzle) into a stage ring; one MMA warp issues
-//     QK^T (A = queries in smem, B = tile K-major) into S in TMEM, and PV with
-//     A = P in TMEM and B = the same smem tile read MN-major; four softmax
-//     warps (one TMEM lane quarter each, one head per thread) read S, apply
-//     the online softmax (rescaling O only when the running max grows by more
-//     than 2^8), and write P (bf16) back over S.
+//   * Per 64-token page: one TMA producer warp loads the page's latent blocks
+//     (128-byte swizzle) into a stage ring, reading page ids a few pages ahead
+//     of the loads; one MMA warp issues QK^T (A = queries in shared memory, B =
+//     tile K-major) into S in TMEM, and PV with A = P in TMEM and B = the same
+//     tile read MN-major; four softmax warps per branch (one TMEM lane quarter
+//     each, one head per thread) read S, apply the online softmax (rescaling O
+//     only when the running max grows by more than 2^8), and write P (bf16)
+//     back over S.
 //   * Rows past the sequence end in the last page are zeroed in shared memory
 //     before the MMAs read them (a NaN there would poison P.V even at P = 0).
-// The split plan, partial-result layout and combine are those of the CUDA-core
-// kernel (slot c + b, running max in log2 units).
+//   * With H <= 32 the query and exchange buffers shrink to 32 rows, which
+//     makes room for a six-page ring.
+//   * Every wait is bounded; a wait that runs out sets the CTA's abort flag and
+//     records MLRA_ERR_TIMEOUT with its site, and every role then leaves.
+// The split plan and the partial-result layout are those of the CUDA-core
+// kernel (slot c + b, running max in log2 units, o_part[slot][H][d_c]).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

@@ -77,9 +77,10 @@ def test_edge_lengths_mla(H, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("H", [128, 32])
 @pytest.mark.parametrize("nbr,bscale", [(2, 0.7), (4, 0.5)])
-def test_mlra_branches(nbr, bscale, kernel):
-    w = synth.workload("mlra4").with_(B=3, seq_len_range=(60, 260), n_branch=nbr, branch_scale=bscale)
+def test_mlra_branches(nbr, bscale, H, kernel):
+    w = synth.workload("mlra4").with_(B=3, H=H, seq_len_range=(60, 260), n_branch=nbr, branch_scale=bscale)
     err, tol, out, ref, _ = run_case(w, kernel)
     assert err <= tol
 
