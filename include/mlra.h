@@ -146,6 +146,26 @@ MLRA_API mlra_status mlra_decode_profiled(const mlra_dims* dims, const void* q_n
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream,
                                  cudaEvent_t* stage_events);
 
+/* mlra_decode_host -- mlra_decode with the step's per-token inputs and its
+ * output in host memory, for a caller whose queries arrive from (and whose
+ * attention output goes back to) the host.  On `stream`, in order: copies
+ * h_q_nope [B,H,d_h], h_q_rope [B,H,d_r], h_q_pos [B] and h_seq_lens [B] into
+ * device staging space inside `workspace`, runs mlra_decode on them, and
+ * copies out [B,H,d_v] to h_out.  Weights, the cache and the page table stay
+ * device-resident (device pointers, as in mla_decode).  The host buffers must
+ * stay valid (and h_out unread) until the stream reaches the end of the call;
+ * pinned host memory makes the copies asynchronous.
+ *   workspace: >= mlra_decode_host_workspace_bytes(dims) bytes, 256-byte
+ *   aligned (the decode workspace followed by the staging space).
+ * The pages specify no host interface; this call only moves the decode's
+ * inputs and output across the host boundary. */
+MLRA_API size_t mlra_decode_host_workspace_bytes(const mlra_dims* dims);
+MLRA_API mlra_status mlra_decode_host(const mlra_dims* dims, const void* h_q_nope, const void* h_q_rope,
+                                      const int32_t* h_q_pos, const void* W_UK, const void* W_UV,
+                                      const void* latent_cache, const void* rope_cache,
+                                      const int32_t* page_table, const int32_t* h_seq_lens, void* h_out,
+                                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Bytes of workspace latent_append needs for hidden width d_model. */
 MLRA_API size_t latent_append_workspace_bytes(const mlra_dims* dims, int d_model);
 

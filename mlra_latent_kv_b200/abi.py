@@ -54,6 +54,8 @@ SIGNATURES = {
     "mla_decode": (ctypes.c_int, _DECODE_ARGS),
     "mlra_decode": (ctypes.c_int, _DECODE_ARGS),
     "mlra_decode_profiled": (ctypes.c_int, _DECODE_ARGS + [_P]),
+    "mlra_decode_host_workspace_bytes": (_SZ, [_DIMS]),
+    "mlra_decode_host": (ctypes.c_int, _DECODE_ARGS),
     "latent_append_workspace_bytes": (_SZ, [_DIMS, ctypes.c_int]),
     "latent_append": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "latent_store": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _I32P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
@@ -140,6 +142,20 @@ def mlra_decode_profiled(dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, 
     arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
     _decode(lib().mlra_decode_profiled, dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache,
             page_table, seq_lens, out, workspace, workspace_nbytes, stream, extra=(ctypes.cast(arr, _P),))
+
+
+def host_workspace_bytes(dims: Dims) -> int:
+    n = lib().mlra_decode_host_workspace_bytes(ctypes.byref(dims))
+    if n == 0:
+        raise MlraError(1, last_error())
+    return int(n)
+
+
+def mlra_decode_host(dims, h_q_nope, h_q_rope, h_q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table,
+                     h_seq_lens, h_out, workspace, workspace_nbytes=None, stream=None):
+    """Per-step inputs and the output are host (pinned) tensors; the rest is device-resident."""
+    _decode(lib().mlra_decode_host, dims, h_q_nope, h_q_rope, h_q_pos, W_UK, W_UV, latent_cache, rope_cache,
+            page_table, h_seq_lens, h_out, workspace, workspace_nbytes, stream)
 
 
 def append_workspace_bytes(dims: Dims, d_model: int) -> int:

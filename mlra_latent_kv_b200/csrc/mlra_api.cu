@@ -251,6 +251,76 @@ mlra_status mlra_decode_profiled(const mlra_dims* dims, const void* q_nope, cons
                      out, workspace, workspace_bytes, stream, stage_events);
 }
 
+// Device staging space for mlra_decode_host, after the decode workspace:
+// q_nope | q_rope | q_pos | seq_lens | out, each 256-byte aligned.
+struct HostStaging {
+  size_t q_nope, q_rope, q_pos, seq_lens, out, total;
+};
+
+static bool host_staging(const mlra_dims* d, const DecodePlan& p, HostStaging* h) {
+  const size_t e = d->dtype == MLRA_BF16 ? 2 : 4;
+  size_t off = round_up(p.total, 256);
+  h->q_nope = off;
+  off = round_up(off + (size_t)d->B * d->H * d->d_h * e, 256);
+  h->q_rope = off;
+  off = round_up(off + (size_t)d->B * d->H * d->d_r * e, 256);
+  h->q_pos = off;
+  off = round_up(off + (size_t)d->B * 4, 256);
+  h->seq_lens = off;
+  off = round_up(off + (size_t)d->B * 4, 256);
+  h->out = off;
+  off = round_up(off + (size_t)d->B * d->H * d->d_v * e, 256);
+  h->total = off;
+  return true;
+}
+
+size_t mlra_decode_host_workspace_bytes(const mlra_dims* dims) {
+  DecodePlan p;
+  if (make_plan(dims, &p) != MLRA_OK) return 0;
+  HostStaging h;
+  host_staging(dims, p, &h);
+  return h.total;
+}
+
+mlra_status mlra_decode_host(const mlra_dims* dims, const void* h_q_nope, const void* h_q_rope,
+                             const int32_t* h_q_pos, const void* W_UK, const void* W_UV, const void* latent_cache,
+                             const void* rope_cache, const int32_t* page_table, const int32_t* h_seq_lens,
+                             void* h_out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  DecodePlan p;
+  mlra_status st = make_plan(dims, &p);
+  if (st != MLRA_OK) return st;
+  if (!h_q_nope || !h_q_rope || !h_q_pos || !h_seq_lens || !h_out)
+    return fail(MLRA_ERR_INVALID_ARG, "a host buffer is NULL");
+  if (!workspace || !aligned(workspace, 256)) return fail(MLRA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  HostStaging h;
+  host_staging(dims, p, &h);
+  if (workspace_bytes < h.total)
+    return fail(MLRA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, h.total);
+  const mlra_dims* d = dims;
+  const size_t e = d->dtype == MLRA_BF16 ? 2 : 4;
+  char* ws = static_cast<char*>(workspace);
+  struct Copy {
+    void* dst;
+    const void* src;
+    size_t n;
+  } in[] = {{ws + h.q_nope, h_q_nope, (size_t)d->B * d->H * d->d_h * e},
+            {ws + h.q_rope, h_q_rope, (size_t)d->B * d->H * d->d_r * e},
+            {ws + h.q_pos, h_q_pos, (size_t)d->B * 4},
+            {ws + h.seq_lens, h_seq_lens, (size_t)d->B * 4}};
+  for (const Copy& c : in) {
+    cudaError_t e2 = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, stream);
+    if (e2 != cudaSuccess) return cuda_fail(e2, "host-to-device copy");
+  }
+  st = decode_impl(d, false, ws + h.q_nope, ws + h.q_rope, reinterpret_cast<const int32_t*>(ws + h.q_pos), W_UK,
+                   W_UV, latent_cache, rope_cache, page_table, reinterpret_cast<const int32_t*>(ws + h.seq_lens),
+                   ws + h.out, workspace, workspace_bytes, stream, nullptr);
+  if (st != MLRA_OK) return st;
+  cudaError_t e3 = cudaMemcpyAsync(h_out, ws + h.out, (size_t)d->B * d->H * d->d_v * e, cudaMemcpyDeviceToHost,
+                                   stream);
+  if (e3 != cudaSuccess) return cuda_fail(e3, "device-to-host copy");
+  return MLRA_OK;
+}
+
 size_t latent_append_workspace_bytes(const mlra_dims* dims, int d_model) {
   if (check_dims(dims) != MLRA_OK) return 0;
   if (d_model < 1) {

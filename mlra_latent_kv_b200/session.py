@@ -93,6 +93,13 @@ class DecodeSession:
                             self.latent_cache, self.rope_cache, self.page_table, self.seq_lens, self.out,
                             self.workspace, stream=stream)
 
+    def decode_host(self, h_q_nope, h_q_rope, h_q_pos, h_seq_lens, h_out, stream=None):
+        """One decode through the host-buffer entry point (inputs in, output out, on `stream`)."""
+        if getattr(self, "host_ws", None) is None:
+            self.host_ws = torch.zeros(abi.host_workspace_bytes(self.dims), dtype=torch.uint8, device=self.device)
+        abi.mlra_decode_host(self.dims, h_q_nope, h_q_rope, h_q_pos, self.W_UK, self.W_UV, self.latent_cache,
+                             self.rope_cache, self.page_table, h_seq_lens, h_out, self.host_ws, stream=stream)
+
     def step(self, stream=None, events=None):
         """One decode step: append the new token (if the workload does), then attend."""
         if self.appends:
@@ -102,6 +109,8 @@ class DecodeSession:
 
     def check(self):
         abi.check_status(self.workspace)
+        if getattr(self, "host_ws", None) is not None:
+            abi.check_status(self.host_ws)
         if self.appends:
             abi.check_status(self.app_ws)
 

@@ -69,6 +69,27 @@ def test_workspace_layout_formula(L):
     assert abi.workspace_bytes(d) == exp
 
 
+def test_host_workspace_layout_formula(L):
+    # decode workspace, then staging: q_nope | q_rope | q_pos | seq_lens | out, each rounded to 256 bytes
+    d = _dims(dtype="f32", kernel="simt", num_splits=10, B=3, H=8, d_h=32, d_v=32, d_c=64, d_r=16)
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    exp = abi.workspace_bytes(d)
+    for n in (3 * 8 * 32 * 4, 3 * 8 * 16 * 4, 3 * 4, 3 * 4, 3 * 8 * 32 * 4):
+        exp = r(exp + n)
+    assert abi.host_workspace_bytes(d) == exp
+
+
+def test_host_decode_validation(L):
+    d = _dims(dtype="f32", kernel="simt", num_splits=10, B=3, H=8, d_h=32, d_v=32, d_c=64, d_r=16)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    st = L.mlra_decode_host(ctypes.byref(d), None, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                            abi.host_workspace_bytes(d), None)
+    assert st == 1 and "host buffer" in abi.last_error()
+    st = L.mlra_decode_host(ctypes.byref(d), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                            abi.host_workspace_bytes(d) - 1, None)
+    assert st == 3
+
+
 @pytest.mark.parametrize("over,status", [
     (dict(d_r=3), 1), (dict(B=0), 1), (dict(n_branch=3), 1), (dict(dtype="bf16", page_size=32), 2),
     (dict(d_c=520), 2), (dict(d_r=128), 2), (dict(softmax_scale=-1.0), 1), (dict(num_pages=0), 1),

@@ -185,3 +185,22 @@ def test_staged_and_graph_launches_bitwise(name):
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
     assert ev[1].elapsed_time(ev[2]) > 0
+
+
+@pytest.mark.parametrize("name", ["dsv2_contiguous", "paged_varlen_h32"])
+def test_host_buffer_decode_bitwise(name):
+    """mlra_decode_host (inputs and output in pinned host memory) gives the same
+    bits as mlra_decode on device copies of the same inputs."""
+    w = synth.workload(name).with_(B=4, seq_len=700, seq_len_range=None)
+    inp = synth.make_inputs(w)
+    s = DecodeSession(w, inp)
+    ref = s.step().clone()
+    h_out = torch.empty(s.out.shape, dtype=s.out.dtype).pin_memory()
+    h_out.fill_(7)
+    s.out.zero_()
+    s.decode_host(inp["q_nope"].pin_memory(), inp["q_rope"].pin_memory(), inp["q_pos"].pin_memory(),
+                  inp["attn_lens"].pin_memory(), h_out)
+    torch.cuda.synchronize()
+    s.check()
+    assert torch.equal(h_out.view(torch.int16), ref.cpu().view(torch.int16))
+    assert torch.count_nonzero(s.out.view(torch.int16)) == 0  # the device-buffer output was not touched
