@@ -403,7 +403,81 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
       long long t_idle = 0;
       while (g_pv < g_end) {
         bool progressed = false;
-        if (g_pv < g_qk) {
+        // MLRA issues the next QK^T before a ready PV (its softmax is the longer
+        // wait); MLA issues the ready PV first (it frees the stage the next load needs)
+        if constexpr (!kExch) {
+          // QK(g) needs S buffer g % kSB, free once PV(g - kSB) is issued; look
+          // ahead at most two pages past the next PV so that PVs (which free the
+          // stages) are not queued behind a run of QKs
+          if (!progressed && g_qk < g_end && g_qk < g_pv + kSB && g_qk <= g_pv + 2) {
+            const uint32_t st = g_qk % kStages;
+            bool ready = lane == 0 ? mbar_test_wait(smem_u32(&bars->stage_full[st]), (g_qk / kStages) & 1) &&
+                                         (!kExch || mbar_test_wait(smem_u32(&bars->rope_full[g_qk & 1]),
+                                                                   (g_qk >> 1) & 1))
+                                   : false;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (ready) {
+              if (lane == 0) MLRA_TRACE_EV(g_qk, kEvStageSeen);
+              uint8_t* tile = sTile + st * L::kStageBytes;
+              uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + 4 * kTileSlotBytes;
+              const int p = walk.pg0 + (int)(g_qk - g0);
+              const int valid = min(kPage, walk.L - p * kPage);
+              if (valid < kPage) {  // zero the rows past the end of the sequence
+                const int nrow = kPage - valid;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                for (int idx = lane; idx < nrow * 8 * 4; idx += 32) {
+                  const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
+                  *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+                }
+                constexpr int kRopeChunks = L::kRopeRowBytes / 16;
+                for (int idx = lane; idx < nrow * kRopeChunks; idx += 32)
+                  *reinterpret_cast<uint4*>(rope_tile + (valid + idx / kRopeChunks) * L::kRopeRowBytes +
+                                            (idx % kRopeChunks) * 16) = z;
+                fence_proxy_async_smem();
+              }
+              __syncwarp();
+              tc_fence_after();
+              if (lane == 0) {
+                MLRA_TRACE_EV(g_qk, kEvQkStart);
+                // descriptors = per-stage base + compile-time offsets (no per-MMA rebuild)
+                const uint64_t td = sdesc_sw128(smem_u32(tile), 16, 1024);
+                const uint32_t s_base = tmem + S_col(g_qk % kSB, 0);
+  #pragma unroll
+                for (int i = 0; i < kBrPerCta; ++i) {
+  #pragma unroll
+                  for (int j = 0; j < kLatPerBr; ++j) {
+                    const int s = i * kLatPerBr + j;
+  #pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                      const uint64_t bd = td + (uint64_t)((s * kTileSlotBytes + ks * 32) >> 4);
+                      mma_ss(s_base + 64u * i, qd + (uint64_t)((s * kQSlotBytes + ks * 32) >> 4), bd, kIdescQK,
+                             (j | ks) ? 1u : 0u);
+                    }
+                  }
+                  if (kExch) {
+                    const uint64_t trd = sdesc_sw64(smem_u32(rope_tile), 512);
+  #pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                      mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2), trd + (uint64_t)(ks * 2), kIdescQK, 1u);
+                  } else {
+  #pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                      mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2),
+                             td + (uint64_t)((4 * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
+                  }
+                }
+                mma_commit(smem_u32(&bars->s_full[g_qk % kSB]));
+                if (kExch) mma_commit(smem_u32(&bars->rope_empty[g_qk & 1]));
+                MLRA_TRACE_EV(g_qk, kEvQkIssued);
+                if (g_qk + 1 == g_end) mma_commit(smem_u32(&bars->q_empty));  // last read of this Q
+              }
+              __syncwarp();
+              ++g_qk;
+              progressed = true;
+            }
+          }
+        }
+        if (!progressed && g_pv < g_qk) {
           if (!o_ready) {  // the previous piece's O must be drained before the first PV overwrites it
             bool r = lane == 0 ? mbar_test_wait(smem_u32(&bars->o_free), (seg - 1) & 1) : false;
             o_ready = __shfl_sync(0xffffffffu, r, 0);
@@ -437,74 +511,76 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
             }
           }
         }
-        // QK(g) needs S buffer g % kSB, free once PV(g - kSB) is issued; look
-        // ahead at most two pages past the next PV so that PVs (which free the
-        // stages) are not queued behind a run of QKs
-        if (!progressed && g_qk < g_end && g_qk < g_pv + kSB && g_qk <= g_pv + 2) {
-          const uint32_t st = g_qk % kStages;
-          bool ready = lane == 0 ? mbar_test_wait(smem_u32(&bars->stage_full[st]), (g_qk / kStages) & 1) &&
-                                       (!kExch || mbar_test_wait(smem_u32(&bars->rope_full[g_qk & 1]),
-                                                                 (g_qk >> 1) & 1))
-                                 : false;
-          ready = __shfl_sync(0xffffffffu, ready, 0);
-          if (ready) {
-            if (lane == 0) MLRA_TRACE_EV(g_qk, kEvStageSeen);
-            uint8_t* tile = sTile + st * L::kStageBytes;
-            uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + 4 * kTileSlotBytes;
-            const int p = walk.pg0 + (int)(g_qk - g0);
-            const int valid = min(kPage, walk.L - p * kPage);
-            if (valid < kPage) {  // zero the rows past the end of the sequence
-              const int nrow = kPage - valid;
-              const uint4 z = make_uint4(0, 0, 0, 0);
-              for (int idx = lane; idx < nrow * 8 * 4; idx += 32) {
-                const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
-                *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+        if constexpr (kExch) {
+          // QK(g) needs S buffer g % kSB, free once PV(g - kSB) is issued; look
+          // ahead at most two pages past the next PV so that PVs (which free the
+          // stages) are not queued behind a run of QKs
+          if (!progressed && g_qk < g_end && g_qk < g_pv + kSB && g_qk <= g_pv + 2) {
+            const uint32_t st = g_qk % kStages;
+            bool ready = lane == 0 ? mbar_test_wait(smem_u32(&bars->stage_full[st]), (g_qk / kStages) & 1) &&
+                                         (!kExch || mbar_test_wait(smem_u32(&bars->rope_full[g_qk & 1]),
+                                                                   (g_qk >> 1) & 1))
+                                   : false;
+            ready = __shfl_sync(0xffffffffu, ready, 0);
+            if (ready) {
+              if (lane == 0) MLRA_TRACE_EV(g_qk, kEvStageSeen);
+              uint8_t* tile = sTile + st * L::kStageBytes;
+              uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + 4 * kTileSlotBytes;
+              const int p = walk.pg0 + (int)(g_qk - g0);
+              const int valid = min(kPage, walk.L - p * kPage);
+              if (valid < kPage) {  // zero the rows past the end of the sequence
+                const int nrow = kPage - valid;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                for (int idx = lane; idx < nrow * 8 * 4; idx += 32) {
+                  const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
+                  *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+                }
+                constexpr int kRopeChunks = L::kRopeRowBytes / 16;
+                for (int idx = lane; idx < nrow * kRopeChunks; idx += 32)
+                  *reinterpret_cast<uint4*>(rope_tile + (valid + idx / kRopeChunks) * L::kRopeRowBytes +
+                                            (idx % kRopeChunks) * 16) = z;
+                fence_proxy_async_smem();
               }
-              constexpr int kRopeChunks = L::kRopeRowBytes / 16;
-              for (int idx = lane; idx < nrow * kRopeChunks; idx += 32)
-                *reinterpret_cast<uint4*>(rope_tile + (valid + idx / kRopeChunks) * L::kRopeRowBytes +
-                                          (idx % kRopeChunks) * 16) = z;
-              fence_proxy_async_smem();
-            }
-            __syncwarp();
-            tc_fence_after();
-            if (lane == 0) {
-              MLRA_TRACE_EV(g_qk, kEvQkStart);
-              // descriptors = per-stage base + compile-time offsets (no per-MMA rebuild)
-              const uint64_t td = sdesc_sw128(smem_u32(tile), 16, 1024);
-              const uint32_t s_base = tmem + S_col(g_qk % kSB, 0);
-#pragma unroll
-              for (int i = 0; i < kBrPerCta; ++i) {
-#pragma unroll
-                for (int j = 0; j < kLatPerBr; ++j) {
-                  const int s = i * kLatPerBr + j;
-#pragma unroll
-                  for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bd = td + (uint64_t)((s * kTileSlotBytes + ks * 32) >> 4);
-                    mma_ss(s_base + 64u * i, qd + (uint64_t)((s * kQSlotBytes + ks * 32) >> 4), bd, kIdescQK,
-                           (j | ks) ? 1u : 0u);
+              __syncwarp();
+              tc_fence_after();
+              if (lane == 0) {
+                MLRA_TRACE_EV(g_qk, kEvQkStart);
+                // descriptors = per-stage base + compile-time offsets (no per-MMA rebuild)
+                const uint64_t td = sdesc_sw128(smem_u32(tile), 16, 1024);
+                const uint32_t s_base = tmem + S_col(g_qk % kSB, 0);
+  #pragma unroll
+                for (int i = 0; i < kBrPerCta; ++i) {
+  #pragma unroll
+                  for (int j = 0; j < kLatPerBr; ++j) {
+                    const int s = i * kLatPerBr + j;
+  #pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                      const uint64_t bd = td + (uint64_t)((s * kTileSlotBytes + ks * 32) >> 4);
+                      mma_ss(s_base + 64u * i, qd + (uint64_t)((s * kQSlotBytes + ks * 32) >> 4), bd, kIdescQK,
+                             (j | ks) ? 1u : 0u);
+                    }
+                  }
+                  if (kExch) {
+                    const uint64_t trd = sdesc_sw64(smem_u32(rope_tile), 512);
+  #pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                      mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2), trd + (uint64_t)(ks * 2), kIdescQK, 1u);
+                  } else {
+  #pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                      mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2),
+                             td + (uint64_t)((4 * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
                   }
                 }
-                if (kExch) {
-                  const uint64_t trd = sdesc_sw64(smem_u32(rope_tile), 512);
-#pragma unroll
-                  for (int ks = 0; ks < 2; ++ks)
-                    mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2), trd + (uint64_t)(ks * 2), kIdescQK, 1u);
-                } else {
-#pragma unroll
-                  for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2),
-                           td + (uint64_t)((4 * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
-                }
+                mma_commit(smem_u32(&bars->s_full[g_qk % kSB]));
+                if (kExch) mma_commit(smem_u32(&bars->rope_empty[g_qk & 1]));
+                MLRA_TRACE_EV(g_qk, kEvQkIssued);
+                if (g_qk + 1 == g_end) mma_commit(smem_u32(&bars->q_empty));  // last read of this Q
               }
-              mma_commit(smem_u32(&bars->s_full[g_qk % kSB]));
-              if (kExch) mma_commit(smem_u32(&bars->rope_empty[g_qk & 1]));
-              MLRA_TRACE_EV(g_qk, kEvQkIssued);
-              if (g_qk + 1 == g_end) mma_commit(smem_u32(&bars->q_empty));  // last read of this Q
+              __syncwarp();
+              ++g_qk;
+              progressed = true;
             }
-            __syncwarp();
-            ++g_qk;
-            progressed = true;
           }
         }
         if (progressed) {
