@@ -225,6 +225,16 @@ MLRA_API mlra_status latent_append_noalloc(const mlra_dims* dims, int d_model, c
                                            const int32_t* page_table, void* latent_cache,
                                            void* rope_cache, cudaStream_t stream);
 
+/* mlra_selftest_wait_timeout -- failure-detection self-test.  Launches one
+ * small kernel on `stream` that waits on a device barrier nothing completes,
+ * using the same bounded wait as every kernel of the library but with a limit
+ * of limit_cycles SM clocks (in [1, 4e9]); the wait gives up, records
+ * MLRA_ERR_TIMEOUT in the error record at the start of `workspace` (>= 256
+ * bytes, zero-filled) and the kernel returns, so the context stays usable.
+ * Read the result with mlra_check_status().  The pages have no counterpart:
+ * this exists to test failure detection without hanging a GPU. */
+MLRA_API mlra_status mlra_selftest_wait_timeout(void* workspace, long long limit_cycles, cudaStream_t stream);
+
 /* Synchronises `stream`, reads the device error record in `workspace`, clears
  * it and returns MLRA_OK, MLRA_ERR_DEVICE_CHECK or MLRA_ERR_TIMEOUT (the
  * message, with the first offending index, goes to mlra_last_error()). */

@@ -61,6 +61,7 @@ SIGNATURES = {
     "latent_store": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _I32P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "latent_append_noalloc": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P]),
     "mlra_check_status": (ctypes.c_int, [_P, _P]),
+    "mlra_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_longlong, _P]),
     "mlra_last_error": (ctypes.c_char_p, []),
     "mlra_shutdown": (None, []),
     "mlra_version": (ctypes.c_int, []),
@@ -192,6 +193,11 @@ def latent_append_noalloc(dims, d_model, h, W_DKV, W_KR, pos, page_table, latent
 
 def check_status(workspace, stream=None) -> None:
     _check(lib().mlra_check_status(_ptr(workspace), _stream(stream)))
+
+
+def selftest_wait_timeout(workspace, limit_cycles: int, stream=None) -> None:
+    """Runs the bounded-wait self-test kernel (see include/mlra.h); read the outcome with check_status."""
+    _check(lib().mlra_selftest_wait_timeout(_ptr(workspace), int(limit_cycles), _stream(stream)))
 
 
 def version() -> int:

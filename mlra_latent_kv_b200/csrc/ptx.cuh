@@ -87,13 +87,13 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err,
-                                          int site) {
+                                          int site, long long limit = kWaitCycles) {
   if (kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       report_error(err, kErrTimeout, site, (int)blockIdx.x);
       return false;

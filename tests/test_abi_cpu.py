@@ -140,3 +140,8 @@ def test_append_and_store_validation(L):
     assert st == 1
     st = L.latent_store(ctypes.byref(d), 10, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None)
     assert st == 1
+
+
+def test_selftest_validation(L):
+    assert L.mlra_selftest_wait_timeout(None, 1000, None) == 1
+    assert L.mlra_selftest_wait_timeout(1 << 20, 0, None) == 1

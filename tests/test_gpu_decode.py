@@ -204,3 +204,17 @@ def test_host_buffer_decode_bitwise(name):
     s.check()
     assert torch.equal(h_out.view(torch.int16), ref.cpu().view(torch.int16))
     assert torch.count_nonzero(s.out.view(torch.int16)) == 0  # the device-buffer output was not touched
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A device wait on a barrier nothing completes gives up after its limit,
+    is reported as MLRA_ERR_TIMEOUT, and later work on the context runs."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    abi.selftest_wait_timeout(ws, 20_000_000)  # ~10 ms of SM clocks
+    with pytest.raises(abi.MlraError) as ei:
+        abi.check_status(ws)
+    assert ei.value.status == 6 and "site 99" in str(ei.value)
+    abi.check_status(ws)  # the record was cleared
+    w = synth.workload("dsv2_contiguous").with_(B=2, seq_len=130)
+    err, tol, *_ = run_case(w, "auto")
+    assert err <= tol
