@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------------------------------
 // a4 + a5: split combine fused into the output up-projection.
-// grid (H, d_v / 128), block 256.
+// grid (H, d_v / 128), block 512.
 //   A (M = 128 value dims, K = d_c) = W_UV[h][:, m0:m0+128]   MN-major (TMA)
 //   B (N = Bp batch rows, K = d_c)  = o_lat[:, h, :] built here in smem:
 //       o_lat[b, h, br cols] = branch_scale * sum_s 2^(m_s - M) o_s / L
