@@ -126,11 +126,11 @@ struct Layout {
 // of each role's events for the first kTracePages pages of CTAs 0 and 1.
 #ifdef MLRA_TRACE
 constexpr int kTracePages = 64;
-constexpr int kTraceEvents = 12;
+constexpr int kTraceEvents = 16;
 __device__ unsigned long long g_trace[2][kTracePages][kTraceEvents];
 __device__ unsigned long long g_span[1024][2];  // entry and exit stamp of every CTA
 enum { kEvTma = 0, kEvStageSeen, kEvQkIssued, kEvSReady, kEvSent, kEvRecv, kEvPReady, kEvPvIssued, kEvMath,
-       kEvSoftmaxDone, kEvQkStart, kEvRecvAdded };
+       kEvSoftmaxDone, kEvQkStart, kEvRecvAdded, kEvXLoaded, kEvXEmptySeen, kEvOwnLoaded, kEvXFullWait };
 #define MLRA_TRACE_EV(gg, ev)                                                                  \
   do {                                                                                         \
     if (blockIdx.x < 2 && (gg) < (uint32_t)kTracePages) g_trace[blockIdx.x][gg][ev] = globaltimer_ns(); \
@@ -635,6 +635,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
           // softmax warp's wait for page g then sees at most one phase ahead
           // (page g + kSB needs QK(g + kSB), hence P(g) written).
           if (lane == 0) mbar_arrive(smem_u32(&bars->xs_read[q4][g % kSB]));
+          if (row == 0) MLRA_TRACE_EV(g, kEvXLoaded);
           uint32_t h[32];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -647,6 +648,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
             ok = false;
             break;
           }
+          if (row == 0) MLRA_TRACE_EV(g, kEvXEmptySeen);
           if (real) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -694,6 +696,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
         }
         if (kExch && warp_real) {
           // s = f16(mine) + f16(peer's): the same bits on both CTAs of the pair
+          if (row == 0) MLRA_TRACE_EV(g, kEvXFullWait);
           if (!mbar_wait_warp<true>(smem_u32(&bars->x_full[q4]), g & 1, abort_flag, err, kSiteXFull)) {
             ok = false;
             break;
