@@ -5,6 +5,8 @@
 // token's K/V information is compressed into c_KV = h W_DKV, the only thing the
 // cache keeps of it; section "2. 解耦旋轉位置編碼": the positional key
 // k_rope = RoPE(h W_KR) is kept beside it without compression.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -13,57 +15,103 @@ namespace mlra {
 // ---------------------------------------------------------------------------
 // latent_append, pass 1: split-K partial products
 //   part[ks, b, j] = sum_{k in chunk ks} h[b, k] * Wcat[k, j],   Wcat = [W_DKV | W_KR]
-// grid (KS), block = one thread per column pair (2j, 2j+1); 64 rows per chunk.
-// Weight rows are read once (the weights dominate the bytes); batch rows are
-// processed 8 at a time from shared memory.
+// grid (KS) chunks of 64 weight rows.  A thread owns kCG adjacent columns (one
+// 16-byte load per weight row) in one of kRG row groups (rows rg, rg + kRG,
+// ...), issues all its row loads before using them, and the row groups are
+// summed in a fixed order through shared memory.  Batch rows are taken kAppendB
+// at a time from shared memory.  Weight rows are read exactly once.
 // ---------------------------------------------------------------------------
 constexpr int kAppendRows = 64;
-constexpr int kAppendB = 8;
+constexpr int kAppendB = 4;
+constexpr int kMaxAppendCols = 512 + 64;  // d_c + d_r at most
+// row groups: 4 with 16-byte column groups, 2 with narrower ones (<= 576 threads)
+template <int kCG>
+constexpr int row_groups() { return kCG >= 4 ? 4 : 2; }
+template <int kCG>
+constexpr int append_threads() { return kMaxAppendCols / kCG * row_groups<kCG>(); }
 
-template <typename T>
-__global__ void append_partial_kernel(const T* __restrict__ h, const T* __restrict__ W_DKV,
+template <typename T, int kCG>
+__global__ void __launch_bounds__(append_threads<kCG>()) append_partial_kernel(const T* __restrict__ h, const T* __restrict__ W_DKV,
                                       const T* __restrict__ W_KR, float* __restrict__ part, AppendArgs a) {
-  __shared__ float hs[kAppendB * kAppendRows];
+  constexpr int kRG = row_groups<kCG>();
+  constexpr int kRowsPerRG = kAppendRows / kRG;
+  extern __shared__ float smem_f[];
+  float* hs = smem_f;                          // [kAppendB][kAppendRows]
+  float* red = smem_f + kAppendB * kAppendRows;  // [kRG - 1][n_cg][kCG][kAppendB]
   const int ks = blockIdx.x;
   const int k0 = ks * kAppendRows;
   const int nk = min(kAppendRows, a.D - k0);
   const int W = a.d_c + a.d_r;
-  const int j = 2 * threadIdx.x;
-  const T* wp = nullptr;
-  int ld = 0;
+  const int n_cg = W / kCG;
+  const int cg = threadIdx.x % n_cg, rg = threadIdx.x / n_cg;
+  const int j = cg * kCG;
+  const T* wp;
+  int ld;
   if (j < a.d_c) {
     wp = W_DKV + j;
     ld = a.d_c;
-  } else if (j < W) {
+  } else {
     wp = W_KR + (j - a.d_c);
     ld = a.d_r;
   }
+  using Vec = typename std::conditional<kCG * sizeof(T) == 16, uint4, typename std::conditional<kCG * sizeof(T) == 8, uint2, uint32_t>::type>::type;
   for (int b0 = 0; b0 < a.B; b0 += kAppendB) {
     for (int e = threadIdx.x; e < kAppendB * kAppendRows; e += blockDim.x) {
       const int bi = e / kAppendRows, k = e % kAppendRows;
       hs[e] = (k < nk && b0 + bi < a.B) ? to_f(h[(size_t)(b0 + bi) * a.D + k0 + k]) : 0.f;
     }
     __syncthreads();
-    if (j < W) {
-      float acc0[kAppendB], acc1[kAppendB];
+    float acc[kCG][kAppendB];
 #pragma unroll
-      for (int i = 0; i < kAppendB; ++i) acc0[i] = acc1[i] = 0.f;
-      const T* wk = wp + (size_t)k0 * ld;
-      for (int k = 0; k < nk; ++k) {
-        const float w0 = to_f(wk[(size_t)k * ld]);
-        const float w1 = to_f(wk[(size_t)k * ld + 1]);
+    for (int c = 0; c < kCG; ++c)
 #pragma unroll
-        for (int i = 0; i < kAppendB; ++i) {
-          const float hv = hs[i * kAppendRows + k];
-          acc0[i] = fmaf(hv, w0, acc0[i]);
-          acc1[i] = fmaf(hv, w1, acc1[i]);
+      for (int i = 0; i < kAppendB; ++i) acc[c][i] = 0.f;
+    constexpr int kBatch = 8;  // weight rows in flight per thread
+#pragma unroll 1
+    for (int r0 = 0; r0 < kRowsPerRG; r0 += kBatch) {
+      Vec wv[kBatch];
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int k = rg + kRG * (r0 + r);
+        if (k < nk) wv[r] = *reinterpret_cast<const Vec*>(wp + (size_t)(k0 + k) * ld);
+      }
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        const int k = rg + kRG * (r0 + r);
+        if (k < nk) {
+          const T* w = reinterpret_cast<const T*>(&wv[r]);
+#pragma unroll
+          for (int c = 0; c < kCG; ++c) {
+            const float wc = to_f(w[c]);
+#pragma unroll
+            for (int i = 0; i < kAppendB; ++i) acc[c][i] = fmaf(hs[i * kAppendRows + k], wc, acc[c][i]);
+          }
         }
+      }
+    }
+    // row groups 1.. hand their sums to row group 0, which adds them in order
+    if (rg > 0) {
+      float* dst = red + ((size_t)(rg - 1) * n_cg + cg) * kCG * kAppendB;
+#pragma unroll
+      for (int c = 0; c < kCG; ++c)
+#pragma unroll
+        for (int i = 0; i < kAppendB; ++i) dst[c * kAppendB + i] = acc[c][i];
+    }
+    __syncthreads();
+    if (rg == 0) {
+      for (int g = 1; g < kRG; ++g) {
+        const float* src = red + ((size_t)(g - 1) * n_cg + cg) * kCG * kAppendB;
+#pragma unroll
+        for (int c = 0; c < kCG; ++c)
+#pragma unroll
+          for (int i = 0; i < kAppendB; ++i) acc[c][i] += src[c * kAppendB + i];
       }
 #pragma unroll
       for (int i = 0; i < kAppendB; ++i) {
         if (b0 + i < a.B) {
-          float2* dst = reinterpret_cast<float2*>(part + ((size_t)ks * a.B + b0 + i) * W + j);
-          *dst = make_float2(acc0[i], acc1[i]);
+          float* dst = part + ((size_t)ks * a.B + b0 + i) * W + j;
+#pragma unroll
+          for (int c = 0; c < kCG; ++c) dst[c] = acc[c][i];
         }
       }
     }
@@ -72,9 +120,11 @@ __global__ void append_partial_kernel(const T* __restrict__ h, const T* __restri
 }
 
 // ---------------------------------------------------------------------------
-// latent_append, pass 2: sum the chunks in order, rotate the RoPE part at
-// pos[b], round once and store into the page slot of position pos[b].
-// One thread per (b, column pair).
+// latent_append, pass 2: sum the chunks, rotate the RoPE part at pos[b],
+// round once and store into the page slot of position pos[b].
+// One warp per (b, column pair): lane l adds chunks l, l + 32, ... in order,
+// then a fixed butterfly adds the lanes (lane 0's result is used), so the sum
+// has the same order on every call.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void append_finalize_kernel(const float* __restrict__ part, const int* __restrict__ pos,
@@ -82,15 +132,31 @@ __global__ void append_finalize_kernel(const float* __restrict__ part, const int
                                        int* __restrict__ err, AppendArgs a, RopeTable tab) {
   const int W = a.d_c + a.d_r;
   const int pairs = W / 2;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int idx = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (idx >= a.B * pairs) return;
   const int b = idx / pairs, j = 2 * (idx % pairs);
   float x0 = 0.f, x1 = 0.f;
-  for (int ks = 0; ks < a.KS; ++ks) {
-    const float2 v = *reinterpret_cast<const float2*>(part + ((size_t)ks * a.B + b) * W + j);
-    x0 += v.x;
-    x1 += v.y;
+  float2 v[4];
+  for (int base = 0; base < a.KS; base += 128) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int ks = base + lane + 32 * u;
+      v[u] = ks < a.KS ? *reinterpret_cast<const float2*>(part + ((size_t)ks * a.B + b) * W + j)
+                       : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      x0 += v[u].x;
+      x1 += v[u].y;
+    }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    x0 += __shfl_xor_sync(0xffffffffu, x0, off);
+    x1 += __shfl_xor_sync(0xffffffffu, x1, off);
+  }
+  if (lane != 0) return;
   const int p = __ldg(pos + b);
   if (p < 0 || p >= a.maxp * kPage) {
     report_error(err, kErrDeviceCheck, b, p);
@@ -110,24 +176,38 @@ __global__ void append_finalize_kernel(const float* __restrict__ part, const int
   }
 }
 
+template <typename T, int kCG>
+static cudaError_t launch_append_t(const void* h, const void* W_DKV, const void* W_KR, const int* pos,
+                                   const int* page_table, void* lat, void* rop, float* part, int* err,
+                                   const AppendArgs& a, const RopeTable& tab, cudaStream_t st) {
+  constexpr int kRG = row_groups<kCG>();
+  const int W = a.d_c + a.d_r;
+  const int n_cg = W / kCG;
+  const int thr = n_cg * kRG;
+  const size_t smem = sizeof(float) * ((size_t)kAppendB * kAppendRows + (size_t)(kRG - 1) * n_cg * kCG * kAppendB);
+  auto k1 = append_partial_kernel<T, kCG>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  k1<<<a.KS, thr, smem, st>>>((const T*)h, (const T*)W_DKV, (const T*)W_KR, part, a);
+  const int n2 = a.B * (W / 2);
+  append_finalize_kernel<T><<<(n2 + 7) / 8, 256, 0, st>>>(part, pos, page_table, (T*)lat, (T*)rop, err, a, tab);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_append(int dtype, const void* h, const void* W_DKV, const void* W_KR, const int* pos,
                           const int* page_table, void* lat, void* rop, float* part, int* err, const AppendArgs& a,
                           const RopeTable& tab, cudaStream_t st) {
-  const int W = a.d_c + a.d_r;
-  const int thr = ((W / 2 + 31) / 32) * 32;
-  const int n2 = a.B * (W / 2);
+  // 16-byte weight loads when both blocks split into whole 16-byte groups, else 4-byte pairs
   if (dtype == 1) {
-    append_partial_kernel<__nv_bfloat16><<<a.KS, thr, 0, st>>>(
-        (const __nv_bfloat16*)h, (const __nv_bfloat16*)W_DKV, (const __nv_bfloat16*)W_KR, part, a);
-    append_finalize_kernel<__nv_bfloat16><<<(n2 + 127) / 128, 128, 0, st>>>(
-        part, pos, page_table, (__nv_bfloat16*)lat, (__nv_bfloat16*)rop, err, a, tab);
-  } else {
-    append_partial_kernel<float><<<a.KS, thr, 0, st>>>((const float*)h, (const float*)W_DKV,
-                                                           (const float*)W_KR, part, a);
-    append_finalize_kernel<float><<<(n2 + 127) / 128, 128, 0, st>>>(part, pos, page_table, (float*)lat,
-                                                                     (float*)rop, err, a, tab);
+    if (a.d_c % 8 == 0 && a.d_r % 8 == 0)
+      return launch_append_t<__nv_bfloat16, 8>(h, W_DKV, W_KR, pos, page_table, lat, rop, part, err, a, tab, st);
+    return launch_append_t<__nv_bfloat16, 2>(h, W_DKV, W_KR, pos, page_table, lat, rop, part, err, a, tab, st);
   }
-  return cudaGetLastError();
+  if (a.d_c % 4 == 0 && a.d_r % 4 == 0)
+    return launch_append_t<float, 4>(h, W_DKV, W_KR, pos, page_table, lat, rop, part, err, a, tab, st);
+  return launch_append_t<float, 2>(h, W_DKV, W_KR, pos, page_table, lat, rop, part, err, a, tab, st);
 }
 
 // ---------------------------------------------------------------------------
