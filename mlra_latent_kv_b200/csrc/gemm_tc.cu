@@ -147,7 +147,11 @@ __global__ void __launch_bounds__(128, 1)
     mma_commit(smem_u32(&done_bar));
   }
   GEMM_TRACE(0, 3);
-  if (mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 21)) {
+  // epilogue: q_lat rows staged as bf16 in the (now free) operand space, then
+  // written to q_ws with 16-byte stores (each row's 128 dims are contiguous)
+  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);  // [Bp][128]; the launch sizes smem for it
+  const bool mma_ok = mbar_wait_warp(smem_u32(&done_bar), 0, &abort_flag, err, 21);
+  if (mma_ok) {
     GEMM_TRACE(0, 4);
     tc_fence_after();
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -155,12 +159,16 @@ __global__ void __launch_bounds__(128, 1)
       uint32_t v[32];
       tmem_ld32(tmem + lane_off + cc, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int b = cc + j;
-        if (b < a.B)
-          q_ws[((size_t)b * a.H + h) * (a.d_c + a.d_r) + m0 + warp * 32 + lane] =
-              __float2bfloat16_rn(__uint_as_float(v[j]) * a.q_scale);
-      }
+      for (int j = 0; j < 32; ++j)
+        stage[(size_t)(cc + j) * 128 + warp * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j]) * a.q_scale);
+    }
+  }
+  __syncthreads();
+  if (mma_ok) {
+    for (int idx = threadIdx.x; idx < a.B * 16; idx += blockDim.x) {
+      const int b = idx >> 4, ch = idx & 15;
+      *reinterpret_cast<uint4*>(q_ws + ((size_t)b * a.H + h) * (a.d_c + a.d_r) + m0 + ch * 8) =
+          *reinterpret_cast<const uint4*>(stage + (size_t)b * 128 + ch * 8);
     }
   }
   tc_fence_before();
@@ -424,7 +432,8 @@ cudaError_t launch_absorb_tc(const void* q_nope, const void* q_rope, const int* 
   if (!tmap_2d(&tw, W_UK, (uint64_t)a.d_c, (uint64_t)a.H * a.K, 64, (uint32_t)a.K) ||
       !tmap_3d_batch(&tq, q_nope, (uint64_t)a.K, (uint64_t)a.H, (uint64_t)a.B, (uint32_t)a.Bp))
     return cudaErrorInvalidValue;
-  const int smem = 1024 + 2 * a.K * 128 + (a.K / 64) * a.Bp * 128;
+  const int operands = 2 * a.K * 128 + (a.K / 64) * a.Bp * 128;
+  const int smem = 1024 + (operands > a.Bp * 256 ? operands : a.Bp * 256);  // operands, later the output stage
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(absorb_tc_kernel), smem);
   if (e != cudaSuccess) return e;
   absorb_tc_kernel<<<dim3(a.H, a.d_c / 128), 128, smem, st>>>(tw, tq, (const __nv_bfloat16*)q_rope, q_pos,
