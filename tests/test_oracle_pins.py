@@ -326,8 +326,10 @@ def test_bytes_per_cached_token():
 # ---------------------------------------------------------------------------
 
 def _pins_pass():
+    """True if every pin holds; a planted slip that makes the oracle raise also counts as caught."""
     try:
         test_brute_force_tiny(2, 0.7)
+        test_brute_force_tiny(4, 0.5)
         for c in _golden()["cases"]:
             test_golden_worked_example(c)
         for c in _golden()["rope_cases"]:
@@ -335,7 +337,8 @@ def _pins_pass():
         test_rope_matches_complex_multiplication()
         test_mlra_identical_branches_equal_mla()
         test_softmax_weights_sum_to_one()
-    except AssertionError:
+        test_latent_append_brute_force()
+    except (AssertionError, ValueError, IndexError):
         return False
     return True
 
@@ -367,10 +370,80 @@ def test_planted_mistakes(monkeypatch):
         qn = a[0]
         return orig_attend(*a, softmax_scale=1.0 / math.sqrt(np.asarray(qn).shape[-1]), **k)
 
-    for name, fn in [("rope", rope_wrong_sign), ("rope", rope_half_index),
+    def rope_rotate_half(x, pos, base=10000.0):
+        # pairs (x[i], x[i + d/2]) instead of the interleaved (x[2i], x[2i+1])
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[-1]
+        idx = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])
+        inv = np.argsort(idx)
+        return orig_rope(x[..., inv], pos, base)[..., idx]
+
+    def angles_missing_factor_two(pos, d_r, base=10000.0):
+        # frequencies base**(-i/d_r) instead of base**(-2i/d_r)
+        i = np.arange(d_r // 2, dtype=np.float64)
+        return np.multiply.outer(np.asarray(pos, dtype=np.float64), np.power(float(base), -i / float(d_r)))
+
+    def attend_no_branch_scale(*a, branch_scale=1.0, **k):
+        return orig_attend(*a, branch_scale=1.0, **k)
+
+    def attend_interleaved_branches(q_nope, q_rope, q_pos, W_UK, W_UV, C, K, heads, n_branch=1, **k):
+        # branch br owns latent dims br, br + n, br + 2n, ... instead of one contiguous block
+        d_c = np.asarray(C).shape[1] if np.asarray(C).ndim == 2 and np.asarray(C).shape[0] else W_UV.shape[1]
+        perm = np.concatenate([np.arange(br, d_c, n_branch) for br in range(n_branch)])
+        return orig_attend(q_nope, q_rope, q_pos, np.asarray(W_UK)[:, :, perm], np.asarray(W_UV)[:, perm, :],
+                           np.asarray(C)[:, perm], K, heads, n_branch=n_branch, **k)
+
+    def attend_keys_shifted(q_nope, q_rope, q_pos, W_UK, W_UV, C, K, heads, **k):
+        # cached token t rotated as if it sat at position t + 1
+        K = np.asarray(K, dtype=np.float64)
+        return orig_attend(q_nope, q_rope, q_pos, W_UK, W_UV, C, orig_rope(K, np.ones(K.shape[0])), heads, **k)
+
+    def attend_query_at_length(q_nope, q_rope, q_pos, W_UK, W_UV, C, K, heads, **k):
+        # the query placed at position L (the sequence length) instead of its own q_pos
+        return orig_attend(q_nope, q_rope, float(np.asarray(C).shape[0]), W_UK, W_UV, C, K, heads, **k)
+
+    orig_gather = mla_oracle.gather_rows
+
+    def gather_reversed(slot_index, page_table_row, L, page_size):
+        return orig_gather(slot_index, page_table_row, L, page_size)[::-1]
+
+    def gather_pages_reversed(slot_index, page_table_row, L, page_size):
+        # the sequence's pages walked last to first; offsets within a page kept
+        t = np.arange(L, dtype=np.int64)
+        row = np.asarray(page_table_row, dtype=np.int64)
+        n_pages = (L + page_size - 1) // page_size
+        return slot_index[row[n_pages - 1 - t // page_size], t % page_size]
+
+    orig_slot_index = mla_oracle.build_slot_index
+
+    def slot_index_first_page_only(tok_seq, tok_pos, page_table, num_pages, page_size):
+        pt = np.asarray(page_table).copy()
+        pt[:, 1:] = pt[:, :1]
+        return orig_slot_index(tok_seq, tok_pos, pt, num_pages, page_size)
+
+    orig_append = mla_oracle.latent_append
+
+    def append_rope_next_position(h, W_DKV, W_KR, pos, rope_base=10000.0):
+        return orig_append(h, W_DKV, W_KR, np.asarray(pos) + 1, rope_base)
+
+    def append_unrotated_key(h, W_DKV, W_KR, pos, rope_base=10000.0):
+        c, _, k_raw = orig_append(h, W_DKV, W_KR, pos, rope_base)
+        return c, k_raw, k_raw
+
+    for name, fn in [("rope", rope_wrong_sign), ("rope", rope_half_index), ("rope", rope_rotate_half),
+                     ("rope_angles", angles_missing_factor_two),
                      ("attend_sequence", attend_no_rope),
                      ("attend_sequence", attend_transposed_wuv),
-                     ("attend_sequence", attend_scale_sqrt_dh)]:
+                     ("attend_sequence", attend_scale_sqrt_dh),
+                     ("attend_sequence", attend_no_branch_scale),
+                     ("attend_sequence", attend_interleaved_branches),
+                     ("attend_sequence", attend_keys_shifted),
+                     ("attend_sequence", attend_query_at_length),
+                     ("gather_rows", gather_reversed),
+                     ("gather_rows", gather_pages_reversed),
+                     ("build_slot_index", slot_index_first_page_only),
+                     ("latent_append", append_rope_next_position),
+                     ("latent_append", append_unrotated_key)]:
         with monkeypatch.context() as m:
             m.setattr(mla_oracle, name, fn)
             m.setattr(oracle, name, fn)
