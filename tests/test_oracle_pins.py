@@ -233,6 +233,21 @@ def test_softmax_weights_sum_to_one():
         np.testing.assert_allclose(got[(0, h)], c @ inp["W_UV"][h], rtol=1e-12, atol=1e-13)
 
 
+@pytest.mark.parametrize("n_branch,bscale", [(1, 1.0), (4, 0.5)])
+def test_single_token_closed_form(n_branch, bscale):
+    """L = 1: each branch puts weight 1 on the only token, whatever the query and its position."""
+    rng = np.random.default_rng(14)
+    inp, ps = _rand_case(rng, B=1, H=3, d_h=4, d_c=8, d_v=3, n_branch=n_branch, lens=(1,), branch_scale=bscale)
+    inp["q_nope"] *= 50.0          # large logits change nothing with one token
+    got = oracle.decode(inp, page_size=ps)
+    c = inp["c_kv"][0]
+    d_cb = 8 // n_branch
+    for h in range(3):
+        exp = sum(bscale * c[br * d_cb:(br + 1) * d_cb] @ inp["W_UV"][h][br * d_cb:(br + 1) * d_cb]
+                  for br in range(n_branch))
+        np.testing.assert_allclose(got[(0, h)], exp, rtol=1e-14, atol=1e-15)
+
+
 def test_planted_dominant_key():
     rng = np.random.default_rng(8)
     inp, ps = _rand_case(rng, B=1, H=1, d_h=4, d_c=8, lens=(6,))
