@@ -23,7 +23,11 @@
 //     f16(own) + f16(peer's), so they hold the same bits and compute identical
 //     softmax weights.
 //   * MLRA with 2 or 4 branches: the branches of a CTA are wholly its own, so
-//     the pair never talks; each CTA adds the full rope score to its branches.
+//     the CTAs of a worker never talk; each adds the full rope score to its
+//     branches.  MLRA-4 with more than 32 heads runs four CTAs per worker, one
+//     branch (128 latent dims) each: O then takes 128 TMEM columns and a page
+//     24 KB of shared memory, so two CTAs fit on one SM and each SM runs two
+//     independent page pipelines.
 //   * Per 64-token page: one TMA producer warp loads the page's latent blocks
 //     (128-byte swizzle) into a stage ring, reading page ids a few pages ahead
 //     of the loads; one MMA warp issues QK^T (A = queries in shared memory, B =
@@ -61,15 +65,27 @@ template <bool kExch, int kBrPerCta>
 constexpr int threads_of() { return 64 + 128 * kBrPerCta + (kExch ? 128 : 0); }  // + MLA exchange warps
 constexpr int kTileSlotBytes = 64 * 128;  // 64 tokens x 64 bf16
 constexpr int kMaxStages = 6;
-constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kIdAhead = 8;               // page ids read this many pages before their tile
 constexpr int kIdRing = 16;
 static_assert(kIdRing >= kIdAhead + 2, "id ring holds the ids in flight");
-// TMEM columns: O [0, 256), then a ring of S buffers of 64 columns per branch
-// the CTA owns: four buffers with one branch per CTA, two with two.
-template <int kBrPerCta>
-constexpr int s_bufs() { return kBrPerCta == 1 ? 4 : 2; }
+// CTAs per worker.  2: a pair on two SMs, each CTA owning 256 latent dims
+// (four 64-dim blocks).  4 (MLRA-4): one branch of 128 latent dims per CTA,
+// two CTAs resident per SM, each with half of the SM's TMEM and shared memory.
+template <int kCtas>
+constexpr int lat_slots() { return 8 / kCtas; }  // 64-dim latent blocks per CTA
+template <int kCtas>
+constexpr uint32_t tmem_cols() { return kCtas == 4 ? 256u : 512u; }
+template <int kCtas>
+constexpr int min_blocks() { return kCtas == 4 ? 2 : 1; }
+// TMEM columns: O [0, 64 * lat_slots), then a ring of S buffers of 64 columns
+// per branch the CTA owns (at most four).
+template <int kBrPerCta, int kCtas>
+constexpr int s_bufs() {
+  return ((int)tmem_cols<kCtas>() - 64 * lat_slots<kCtas>()) / (64 * kBrPerCta) < 4
+             ? ((int)tmem_cols<kCtas>() - 64 * lat_slots<kCtas>()) / (64 * kBrPerCta)
+             : 4;
+}
 
 struct Bars {
   uint64_t q_full, q_empty;
@@ -90,36 +106,42 @@ struct Bars {
 //  stages; the CTA's half of the rope dims (32, 64-byte swizzle) in its own
 //  two-slot ring, released as soon as QK^T has read it; one fp16 exchange
 //  buffer for the partial scores of one page.
-//  MLRA: 4 latent blocks + the full rope block (128-byte swizzle) per stage,
-//  ring of 3 stages.
+//  MLRA: the CTA's latent blocks + the full rope block (128-byte swizzle) per
+//  stage; a ring of 3 stages for a pair (4 blocks), 2 for a quad (2 blocks,
+//  two CTAs per SM).
 //  Query blocks, the exchange buffer and the rope query take kHq rows: 128,
 //  or 32 when H <= 32, which leaves room for two more stages.  The M = 128
 //  MMAs read 128 rows from each query block; the rows past kHq fall on the
 //  next buffer, feed only MMA rows of absent heads, and are never used.
-template <bool kExch, int kHq>
+template <bool kExch, int kHq, int kCtas>
 struct Layout {
+  static constexpr int kLat = lat_slots<kCtas>();
+  // per-CTA shared memory: one CTA per SM, or half of the SM's 228 KB less the
+  // 1 KB the hardware reserves per CTA
+  static constexpr int kCap = min_blocks<kCtas>() == 1 ? 232448 : 233472 / 2 - 1024;
   static constexpr int kQSlotBytes = kHq * 128;  // kHq query rows x 64 bf16
   static constexpr int kRopeQBytes = kExch ? kHq * 64 : kQSlotBytes;
   static constexpr int kRopeTileBytes = kExch ? 64 * 64 : kTileSlotBytes;
   static constexpr int kRopeRowBytes = kExch ? 64 : 128;
   static constexpr int kXBytes = 64 * kHq * 2;   // one page of fp16 partial scores, kHq rows
-  static constexpr int kStageBytes = 4 * kTileSlotBytes + (kExch ? 0 : kRopeTileBytes);
+  static constexpr int kStageBytes = kLat * kTileSlotBytes + (kExch ? 0 : kRopeTileBytes);
   static constexpr int kQ = 0;
-  static constexpr int kQRope = 4 * kQSlotBytes;
+  static constexpr int kQRope = kLat * kQSlotBytes;
   static constexpr int kRope = kQRope + kRopeQBytes;  // MLA rope ring
   static constexpr int kX = kRope + (kExch ? 2 * kRopeTileBytes : 0);
   static constexpr int kTile = (kX + (kExch ? kXBytes : 0) + 1023) / 1024 * 1024;
   static constexpr int kFixed = kTile + (int)sizeof(Bars) + 1024;  // + alignment slack
-  static constexpr int kStages = (232448 - kFixed) / kStageBytes < kMaxStages ? (232448 - kFixed) / kStageBytes
-                                                                                : kMaxStages;
+  static constexpr int kStages = (kCap - kFixed) / kStageBytes < kMaxStages ? (kCap - kFixed) / kStageBytes
+                                                                              : kMaxStages;
   static constexpr int kBars = kTile + kStages * kStageBytes;
   static constexpr int kBytes = kBars + (int)sizeof(Bars) + 1024;
-  static_assert(kStages >= 3, "stage ring");
+  static_assert(kStages >= (kCtas == 4 ? 2 : 3), "stage ring");
   static_assert(kStageBytes % 1024 == 0 && kTile % 1024 == 0 && kRope % 512 == 0 && kQRope % 1024 == 0,
                 "aligned slots");
-  static_assert(kBytes <= 232448, "shared memory");
+  static_assert(kBytes <= kCap, "shared memory");
   // the last query block's 128-row MMA read stays inside the CTA's shared memory
-  static_assert(3 * kQSlotBytes + 128 * 128 <= kBytes && kQRope + 128 * (kExch ? 64 : 128) <= kBytes, "query reads");
+  static_assert((kLat - 1) * kQSlotBytes + 128 * 128 <= kBytes && kQRope + 128 * (kExch ? 64 : 128) <= kBytes,
+                "query reads");
 };
 
 // Optional pipeline trace (builds with -DMLRA_TRACE only): globaltimer stamps
@@ -212,16 +234,20 @@ __device__ __forceinline__ bool softmax_page(float (&s)[64], int valid, bool fir
   return rescale;
 }
 
-template <bool kExch, int kBrPerCta, int kHq>
-__global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
+template <bool kExch, int kBrPerCta, int kHq, int kCtas>
+__global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCtas>())
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rope,
                      const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
                      const int* __restrict__ page_table, const int* __restrict__ seq_lens,
                      float* __restrict__ o_part, float* __restrict__ ml_part, int* __restrict__ err, AttnArgs a) {
-  using L = Layout<kExch, kHq>;
+  using L = Layout<kExch, kHq, kCtas>;
   constexpr int kQSlotBytes = L::kQSlotBytes;
-  constexpr int kLatPerBr = 4 / kBrPerCta;      // latent slots per branch
-  constexpr int kPvN = 256 / kBrPerCta;         // PV output columns per branch
+  constexpr int kLat = L::kLat;                 // latent slots of this CTA
+  constexpr int kLatPerBr = kLat / kBrPerCta;   // latent slots per branch
+  constexpr int kOCols = 64 * kLat;             // TMEM columns of O
+  constexpr int kPvN = kOCols / kBrPerCta;      // PV output columns per branch
+  constexpr uint32_t kTmemCols = tmem_cols<kCtas>();
+  static_assert(!kExch || kCtas == 2, "the score exchange is between the two CTAs of a pair");
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kPvN, false, true);
 
@@ -241,8 +267,8 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
 #ifdef MLRA_TRACE
   if (threadIdx.x == 0 && blockIdx.x < 1024) g_span[blockIdx.x][0] = globaltimer_ns();
 #endif
-  const uint32_t rank = kExch ? cluster_ctarank() : (blockIdx.x & 1u);
-  const int c = blockIdx.x >> 1;
+  const uint32_t rank = kExch ? cluster_ctarank() : (blockIdx.x % (unsigned)kCtas);
+  const int c = blockIdx.x / kCtas;
   const int maxL = a.maxp * kPage;
   const int rope_q_bytes = a.H * (kExch ? 64 : 128);  // H query rows of the rope block
 
@@ -295,12 +321,12 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
   const uint32_t tmem = bars->tmem_base;
   const WorkerPlan plan = bars->plan;
 
-  // S ring (kSB buffers of 64 columns per branch) after the 256 columns of O
-  constexpr int kSB = s_bufs<kBrPerCta>();
+  // S ring (kSB buffers of 64 columns per branch) after the columns of O
+  constexpr int kSB = s_bufs<kBrPerCta, kCtas>();
   auto S_col = [](uint32_t buf, int i) -> uint32_t {
-    return 256u + buf * (64u * kBrPerCta) + (uint32_t)i * 64u;
+    return (uint32_t)kOCols + buf * (64u * kBrPerCta) + (uint32_t)i * 64u;
   };
-  static_assert(256 + kSB * 64 * kBrPerCta <= 512, "TMEM columns overflow");
+  static_assert(kSB >= 2 && kOCols + kSB * 64 * kBrPerCta <= (int)kTmemCols, "TMEM columns overflow");
   auto O_col = [](int i) -> uint32_t { return (uint32_t)i * (uint32_t)kPvN; };
 
   if (warp == 0) {
@@ -339,9 +365,9 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
       while (ok && walk.next(seq_lens)) {
         if (seg > 0 && !mbar_wait(smem_u32(&bars->q_empty), (seg - 1) & 1, abort_flag, err, kSiteQEmpty)) break;
         const uint32_t qb = smem_u32(&bars->q_full);
-        mbar_expect_tx(qb, 4 * a.H * 128 + rope_q_bytes);
-        for (int s = 0; s < 4; ++s)
-          tma_load_2d(smem_u32(sQ + s * kQSlotBytes), &tm_q, qb, 64 * (4 * (int)rank + s), walk.b * a.H);
+        mbar_expect_tx(qb, kLat * a.H * 128 + rope_q_bytes);
+        for (int s = 0; s < kLat; ++s)
+          tma_load_2d(smem_u32(sQ + s * kQSlotBytes), &tm_q, qb, 64 * (kLat * (int)rank + s), walk.b * a.H);
         if (kExch)
           tma_load_2d(smem_u32(sQRope), &tm_q_rope, qb, a.d_c + 32 * (int)rank, walk.b * a.H);
         else
@@ -369,14 +395,14 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
           const uint32_t fb = smem_u32(&bars->stage_full[st]);
           uint8_t* tile = sTile + st * L::kStageBytes;
           mbar_expect_tx(fb, L::kStageBytes);
-          for (int s = 0; s < 4; ++s)
-            tma_load_2d(smem_u32(tile + s * kTileSlotBytes), &tm_lat, fb, 64 * (4 * (int)rank + s), pg * kPage);
+          for (int s = 0; s < kLat; ++s)
+            tma_load_2d(smem_u32(tile + s * kTileSlotBytes), &tm_lat, fb, 64 * (kLat * (int)rank + s), pg * kPage);
           if (kExch) {
             const uint32_t rb = smem_u32(&bars->rope_full[g & 1]);
             mbar_expect_tx(rb, L::kRopeTileBytes);
             tma_load_2d(smem_u32(sRope + (g & 1) * L::kRopeTileBytes), &tm_rope, rb, 32 * (int)rank, pg * kPage);
           } else {
-            tma_load_2d(smem_u32(tile + 4 * kTileSlotBytes), &tm_rope, fb, 0, pg * kPage);
+            tma_load_2d(smem_u32(tile + kLat * kTileSlotBytes), &tm_rope, fb, 0, pg * kPage);
           }
           MLRA_TRACE_EV(g, kEvTma);
         }
@@ -419,13 +445,13 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
             if (ready) {
               if (lane == 0) MLRA_TRACE_EV(g_qk, kEvStageSeen);
               uint8_t* tile = sTile + st * L::kStageBytes;
-              uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + 4 * kTileSlotBytes;
+              uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + kLat * kTileSlotBytes;
               const int p = walk.pg0 + (int)(g_qk - g0);
               const int valid = min(kPage, walk.L - p * kPage);
               if (valid < kPage) {  // zero the rows past the end of the sequence
                 const int nrow = kPage - valid;
                 const uint4 z = make_uint4(0, 0, 0, 0);
-                for (int idx = lane; idx < nrow * 8 * 4; idx += 32) {
+                for (int idx = lane; idx < nrow * 8 * kLat; idx += 32) {
                   const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
                   *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
                 }
@@ -463,7 +489,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
   #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                       mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2),
-                             td + (uint64_t)((4 * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
+                             td + (uint64_t)((kLat * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
                   }
                 }
                 mma_commit(smem_u32(&bars->s_full[g_qk % kSB]));
@@ -525,13 +551,13 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
             if (ready) {
               if (lane == 0) MLRA_TRACE_EV(g_qk, kEvStageSeen);
               uint8_t* tile = sTile + st * L::kStageBytes;
-              uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + 4 * kTileSlotBytes;
+              uint8_t* rope_tile = kExch ? sRope + (g_qk & 1) * L::kRopeTileBytes : tile + kLat * kTileSlotBytes;
               const int p = walk.pg0 + (int)(g_qk - g0);
               const int valid = min(kPage, walk.L - p * kPage);
               if (valid < kPage) {  // zero the rows past the end of the sequence
                 const int nrow = kPage - valid;
                 const uint4 z = make_uint4(0, 0, 0, 0);
-                for (int idx = lane; idx < nrow * 8 * 4; idx += 32) {
+                for (int idx = lane; idx < nrow * 8 * kLat; idx += 32) {
                   const int s = idx / (nrow * 8), rem = idx % (nrow * 8);
                   *reinterpret_cast<uint4*>(tile + s * kTileSlotBytes + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
                 }
@@ -569,7 +595,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
   #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                       mma_ss(s_base + 64u * i, qrd + (uint64_t)(ks * 2),
-                             td + (uint64_t)((4 * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
+                             td + (uint64_t)((kLat * kTileSlotBytes + ks * 32) >> 4), kIdescQK, 1u);
                   }
                 }
                 mma_commit(smem_u32(&bars->s_full[g_qk % kSB]));
@@ -780,7 +806,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + O_col(bi) + cc, o);
           if (real) {
-            const int d0 = 256 * (int)rank + (int)O_col(bi) + cc;
+            const int d0 = kOCols * (int)rank + (int)O_col(bi) + cc;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int d = d0 + 8 * q;
@@ -817,17 +843,22 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), 1)
 // ---------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
-template <bool kExch, int kBrPerCta, int kHq>
+template <bool kExch, int kBrPerCta, int kHq, int kCtas>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const CUtensorMap& tl, const CUtensorMap& tr,
                            const int* page_table,
                            const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                            cudaStream_t st, bool pdl) {
-  auto kern = attend_tc_kernel<kExch, kBrPerCta, kHq>;
-  const int smem = Layout<kExch, kHq>::kBytes;
+  auto kern = attend_tc_kernel<kExch, kBrPerCta, kHq, kCtas>;
+  const int smem = Layout<kExch, kHq, kCtas>::kBytes;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
+  if (min_blocks<kCtas>() > 1) {  // the whole unified L1/shared array as shared memory: two CTAs per SM
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributePreferredSharedMemoryCarveout,
+                             100);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * a.G, 1, 1);
+  cfg.gridDim = dim3(kCtas * a.G, 1, 1);
   cfg.blockDim = dim3(threads_of<kExch, kBrPerCta>(), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -866,13 +897,14 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
     tqr = tq;
     if (!tmap_2d(&tr, rop, (uint64_t)a.d_r, (uint64_t)a.num_pages * kPage, 64, 64)) return cudaErrorInvalidValue;
   }
-#define MLRA_LAUNCH(E, BR, HQ) \
-  launch_variant<E, BR, HQ>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl)
+#define MLRA_LAUNCH(E, BR, HQ, CTAS) \
+  launch_variant<E, BR, HQ, CTAS>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl)
   const bool small = a.H <= 32;  // compact query buffers, deeper ring
   switch (a.n_branch) {
-    case 1: return small ? MLRA_LAUNCH(true, 1, 32) : MLRA_LAUNCH(true, 1, 128);
-    case 2: return small ? MLRA_LAUNCH(false, 1, 32) : MLRA_LAUNCH(false, 1, 128);
-    case 4: return small ? MLRA_LAUNCH(false, 2, 32) : MLRA_LAUNCH(false, 2, 128);
+    case 1: return small ? MLRA_LAUNCH(true, 1, 32, 2) : MLRA_LAUNCH(true, 1, 128, 2);
+    case 2: return small ? MLRA_LAUNCH(false, 1, 32, 2) : MLRA_LAUNCH(false, 1, 128, 2);
+    // MLRA-4 at full head count: four one-branch CTAs per worker, two per SM
+    case 4: return small ? MLRA_LAUNCH(false, 2, 32, 2) : MLRA_LAUNCH(false, 1, 128, 4);
     default: return cudaErrorInvalidValue;
   }
 #undef MLRA_LAUNCH
