@@ -58,11 +58,10 @@ def test_reduced_workloads_few_workers(name, G):
     assert err <= tol, f"{name}/G={G}: max err {err:.3e} > tol {tol:.3e}"
 
 
-@pytest.mark.parametrize("kernel", KERNELS)
-@pytest.mark.parametrize("H", [128, 64, 32, 8])
-def test_edge_lengths_mla(H, kernel):
+def _edge_lengths(w, kernel):
+    """Empty, one-token and page-boundary lengths, with NaN in every unused cache slot."""
     lens = [0, 1, 63, 64, 65, 127, 128, 129]
-    w = synth.workload("dsv2_contiguous").with_(B=len(lens), H=H, seq_len_range=(1, 2), paged=True, nan_tails=True)
+    w = w.with_(B=len(lens), seq_len_range=(1, 2), paged=True, nan_tails=True)
     inp = synth.make_inputs(w.with_(seq_len_range=None, seq_len=max(lens)))
     # rebuild with explicit lengths: draw at max length, keep the first L_b tokens of each sequence
     keep = np.concatenate([np.arange(max(lens)) < L for L in lens])
@@ -72,8 +71,20 @@ def test_edge_lengths_mla(H, kernel):
     inp["attn_lens"] = inp["seq_lens"].clone()
     inp["q_pos"] = inp["seq_lens"].clone()
     err, tol, out, ref, _ = run_case(w, kernel, inp=inp)
-    assert err <= tol, f"H={H}/{kernel}: {err:.3e} > {tol:.3e}"
+    assert err <= tol, f"H={w.H}/n_branch={w.n_branch}/{kernel}: {err:.3e} > {tol:.3e}"
     assert torch.all(out[0] == 0), "empty sequence must give a zero row"
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("H", [128, 64, 32, 8])
+def test_edge_lengths_mla(H, kernel):
+    _edge_lengths(synth.workload("dsv2_contiguous").with_(H=H), kernel)
+
+
+@pytest.mark.parametrize("H", [128, 64])
+def test_edge_lengths_mlra4(H):
+    """MLRA-4 above 32 heads runs four one-branch CTAs per worker (two 64-dim latent blocks each)."""
+    _edge_lengths(synth.workload("mlra4").with_(H=H), "auto")
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
