@@ -18,9 +18,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
-import math
 import os
 import statistics
 import sys

@@ -4,7 +4,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from oracle.inputs import f64, oracle_inputs  # noqa: F401
+from oracle.inputs import oracle_inputs  # noqa: F401  (re-exported for the GPU tests)
 
 
 def tolerance(ref_values: np.ndarray) -> float:
