@@ -364,7 +364,8 @@ def run_ours(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
         "ms_per_step": max_total_ms / K, "us_per_step": max_total_ms / K * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded per workload, shapes of the workload configuration)",
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded per workload, shapes of the workload configuration)",
         "config": config_of(w, inp, ws),
         "stage_us": {k: v * 1e3 for k, v in stage_ms.items()},
         "roofline": {"kernel": "split-KV latent attention", "bound": "hbm", "achieved": achieved,
