@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 
 import oracle
+from oracle import inputs as oracle_inputs_mod
 from oracle import mla_oracle
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
@@ -327,6 +328,59 @@ def test_latent_append_brute_force():
         np.testing.assert_allclose(k_rot[b], brute_rope(kb, pos[b], 10000.0), rtol=0, atol=1e-12)
 
 
+def _tiny_append_case():
+    """A step that appends: lengths 63 and 64 put the new token in the last slot
+    of a page and in the first slot of a new page (64-token pages)."""
+    from mlra_latent_kv_b200 import synth
+    w = synth.workload("longctx_append").with_(B=4, H=2, d_h=4, d_v=3, d_c=8, d_r=4, seq_len=None,
+                                               seq_len_range=(62, 64), append_d_model=5, dtype="f32",
+                                               weight_std=0.3, seed=41)
+    inp = synth.make_inputs(w)
+    assert {63, 64} <= set(inp["seq_lens"].tolist())
+    return w, inp
+
+
+def test_oracle_inputs_appends_token_at_its_position():
+    """The oracle's view of an appending step holds each sequence's new token,
+    compressed by brute force, at (sequence b, position pos[b]) with its RAW
+    positional key, and decoding it equals a brute-force decode over L + 1
+    tokens whose last token sits at position pos (yololab.net, sections
+    "1. 鍵值聯合低秩壓縮" and "2. 解耦旋轉位置編碼")."""
+    w, inp = _tiny_append_case()
+    oi = oracle_inputs_mod.oracle_inputs(w, inp)
+    T = inp["c_kv"].shape[0]
+    h, Wd, Wr = (inp[k].double().numpy() for k in ("h", "W_DKV", "W_KR"))
+    pos = inp["pos"].numpy()
+    L = inp["seq_lens"].numpy()
+    np.testing.assert_array_equal(pos, L)                       # the new token follows the cached ones
+    np.testing.assert_array_equal(inp["q_pos"].numpy(), pos)    # and the query sits at its position
+    np.testing.assert_array_equal(oi["seq_lens"], L + 1)
+    np.testing.assert_array_equal(oi["c_kv"][:T], inp["c_kv"].double().numpy())
+    np.testing.assert_array_equal(oi["tok_pos"][:T], inp["tok_pos"].numpy())
+    appended = {}
+    for b in range(w.B):
+        rows = np.where((oi["tok_seq"] == b) & (oi["tok_pos"] == pos[b]))[0]
+        assert len(rows) == 1 and rows[0] >= T
+        c_b = [sum(h[b, k] * Wd[k, j] for k in range(h.shape[1])) for j in range(w.d_c)]
+        k_b = [sum(h[b, k] * Wr[k, j] for k in range(h.shape[1])) for j in range(w.d_r)]
+        np.testing.assert_allclose(oi["c_kv"][rows[0]], c_b, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(oi["k_rope"][rows[0]], k_b, rtol=0, atol=1e-12)
+        appended[b] = (c_b, k_b)
+    got = oracle.decode(oi)
+    scale = 1.0 / math.sqrt(w.d_h + w.d_r)
+    for b in range(w.B):
+        rows = sorted(np.where(inp["tok_seq"].numpy() == b)[0], key=lambda i: int(inp["tok_pos"][i]))
+        C = [list(inp["c_kv"][i].double().numpy()) for i in rows] + [appended[b][0]]
+        K = [list(inp["k_rope"][i].double().numpy()) for i in rows] + [appended[b][1]]
+        assert len(C) == L[b] + 1
+        for hh in range(w.H):
+            ref = brute_decode_one(list(inp["q_nope"][b, hh].double().numpy()),
+                                   list(inp["q_rope"][b, hh].double().numpy()), float(inp["q_pos"][b]),
+                                   inp["W_UK"][hh].double().numpy().tolist(),
+                                   inp["W_UV"][hh].double().numpy().tolist(), C, K, 1, 1.0, scale, w.rope_base)
+            np.testing.assert_allclose(got[(b, hh)], ref, rtol=0, atol=1e-12)
+
+
 def test_bytes_per_cached_token():
     """576 stored dims (512 latent + 64 rope) in bf16 = 1152 B per token."""
     from mlra_latent_kv_b200 import synth
@@ -353,6 +407,7 @@ def _pins_pass():
         test_mlra_identical_branches_equal_mla()
         test_softmax_weights_sum_to_one()
         test_latent_append_brute_force()
+        test_oracle_inputs_appends_token_at_its_position()
     except (AssertionError, ValueError, IndexError):
         return False
     return True
@@ -444,6 +499,27 @@ def test_planted_mistakes(monkeypatch):
     def append_unrotated_key(h, W_DKV, W_KR, pos, rope_base=10000.0):
         c, _, k_raw = orig_append(h, W_DKV, W_KR, pos, rope_base)
         return c, k_raw, k_raw
+
+    orig_inputs = oracle_inputs_mod.oracle_inputs
+
+    def inputs_append_next_position(w, inp):
+        # the appended token placed one position after the one it is written at
+        d = orig_inputs(w, inp)
+        d["tok_pos"] = d["tok_pos"].copy()
+        d["tok_pos"][-w.B:] += 1
+        return d
+
+    def inputs_append_rotated_key(w, inp):
+        # the appended token's positional key kept rotated (the oracle rotates on read)
+        d = orig_inputs(w, inp)
+        d["k_rope"] = d["k_rope"].copy()
+        d["k_rope"][-w.B:] = mla_oracle.rope(d["k_rope"][-w.B:], d["tok_pos"][-w.B:], w.rope_base)
+        return d
+
+    for fn in (inputs_append_next_position, inputs_append_rotated_key):
+        with monkeypatch.context() as m:
+            m.setattr(oracle_inputs_mod, "oracle_inputs", fn)
+            assert not _pins_pass(), f"planted mistake in oracle_inputs ({fn.__name__}) went unnoticed"
 
     for name, fn in [("rope", rope_wrong_sign), ("rope", rope_half_index), ("rope", rope_rotate_half),
                      ("rope_angles", angles_missing_factor_two),
