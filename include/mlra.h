@@ -29,7 +29,11 @@
  *     device (a page id outside [0, num_pages), a bounded wait that gave up)
  *     are recorded in the first 16 bytes of the workspace and read with
  *     mlra_check_status().  The workspace must be zero-filled once before its
- *     first use; mlra_check_status() clears what it reports.
+ *     first use; mlra_check_status() clears what it reports.  A bad page id
+ *     met on a read (decode) is replaced by page 0, so the read stays inside
+ *     the pool and that call's output is void; met on a write (latent_append,
+ *     latent_store, latent_append_noalloc) the token is not written at all,
+ *     so no other sequence's page is touched.
  */
 #ifndef MLRA_H_
 #define MLRA_H_
@@ -166,6 +170,18 @@ MLRA_API mlra_status mlra_decode_host(const mlra_dims* dims, const void* h_q_nop
                                       const int32_t* page_table, const int32_t* h_seq_lens, void* h_out,
                                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* mlra_describe_plan -- the kernels mla_decode / mlra_decode launch for
+ * `dims`, as one NUL-terminated line of ';'-separated key=value fields:
+ *   family     tcgen05 | tcgen05+cuda-core | cuda-core (kernel AUTO picks
+ *              tcgen05 wherever the shape allows; dims.kernel forces one)
+ *   splits     split-KV workers;  kernels  launches per decode call
+ *   absorb, attention, combine, upproj   the kernel of each stage
+ * Touches no GPU memory.  With num_splits = 0 it reads the current device's
+ * SM count (as the decode calls do).  Returns MLRA_ERR_INVALID_ARG when
+ * buf_len is too short.  The pages have no counterpart: this reports which of
+ * the library's own kernels serve the decode step of the method above. */
+MLRA_API mlra_status mlra_describe_plan(const mlra_dims* dims, char* buf, size_t buf_len);
+
 /* Bytes of workspace latent_append needs for hidden width d_model. */
 MLRA_API size_t latent_append_workspace_bytes(const mlra_dims* dims, int d_model);
 
@@ -212,11 +228,22 @@ MLRA_API mlra_status latent_store(const mlra_dims* dims, int n_tokens, const voi
  *     that needs more returns MLRA_ERR_UNSUPPORTED and enqueues nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept per device and
+ *     context; after cudaDeviceReset (or any release of a device's primary
+ *     context) call mlra_shutdown() before the next call, which forgets it.
+ *   - Memory: the array lives in the same device module as every kernel of
+ *     the library, so every process that uses any entry point holds its
+ *     4 MiB on each device it runs on.  Under CUDA's lazy module loading (the
+ *     default) that memory is taken when the library first launches a kernel
+ *     or looks up a symbol on the device, not when it is loaded: an engine
+ *     that reserves all free HBM for its pool should make one call of the
+ *     library (e.g. a first latent_append_noalloc) on each device BEFORE it
+ *     reserves the memory.
  *   - Every call shares the one array.  Each call overwrites the part it uses
  *     before reading it, so nothing has to start zeroed, but calls whose
  *     kernels overlap on the GPU (e.g. on two streams) race on it.
- *   - Device-side range checks still keep every access inside the cache, but
+ *   - Device-side range checks still skip every write whose page id or
+ *     position is out of range (nothing else in the cache changes), but
  *     their reports are not recorded (there is no workspace to hold them).
  * It allocates nothing and frees nothing. */
 #define MLRA_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -243,8 +270,9 @@ MLRA_API mlra_status mlra_check_status(void* workspace, cudaStream_t stream);
 /* Message of the last error on the calling thread ("" if none). */
 MLRA_API const char* mlra_last_error(void);
 
-/* Frees host-side caches (TMA descriptors).  Safe to call at any time when no
- * call is in progress on another thread. */
+/* Frees host-side caches (TMA descriptors, and the device address of
+ * latent_append_noalloc's scratch).  Safe to call at any time when no call is
+ * in progress on another thread. */
 MLRA_API void mlra_shutdown(void);
 
 /* ABI version: 1. */

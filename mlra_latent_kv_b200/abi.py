@@ -60,6 +60,7 @@ SIGNATURES = {
     "latent_append": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "latent_store": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _I32P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "latent_append_noalloc": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P]),
+    "mlra_describe_plan": (ctypes.c_int, [_DIMS, ctypes.c_char_p, _SZ]),
     "mlra_check_status": (ctypes.c_int, [_P, _P]),
     "mlra_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_longlong, _P]),
     "mlra_last_error": (ctypes.c_char_p, []),
@@ -107,6 +108,16 @@ def _stream(stream) -> int | None:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def describe_plan(dims: Dims) -> dict:
+    """The kernels a decode call launches for ``dims`` (family, splits,
+    launches per call, and the kernel of each stage), as the library plans them."""
+    buf = ctypes.create_string_buffer(512)
+    _check(lib().mlra_describe_plan(ctypes.byref(dims), buf, len(buf)))
+    out = dict(kv.split("=", 1) for kv in buf.value.decode().split(";"))
+    out["splits"], out["kernels"] = int(out["splits"]), int(out["kernels"])
+    return out
 
 
 def workspace_bytes(dims: Dims) -> int:

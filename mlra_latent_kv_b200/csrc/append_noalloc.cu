@@ -5,6 +5,9 @@
 // The split-K partial sums that latent_append keeps in the caller's workspace
 // live here in one fixed, file-scope device array instead.  There is no
 // counterpart on the pages.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstdio>
 #include <mutex>
 
@@ -19,31 +22,66 @@ static __device__ __align__(256) unsigned char g_append_scratch[MLRA_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_dev[kMaxDevices] = {};  // device address of g_append_scratch, by device ordinal
+// Device address of g_append_scratch per device ordinal, with the context it
+// was looked up in: a context created later (after cudaDeviceReset, or after
+// the primary context was released and made again) holds the array at a new
+// address, so the entry is looked up again when the current context differs.
+struct ScratchEntry {
+  CUcontext ctx;
+  void* ptr;
+};
+ScratchEntry g_scratch_dev[kMaxDevices] = {};
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;  // the driver's cuCtxGetCurrent, looked up through the runtime
+
+// The calling thread's current context, or nullptr if there is none (or the
+// driver function cannot be had, in which case the cache is used per device).
+CUcontext current_context() {
+  if (g_ctx_current == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }
+  CUcontext ctx = nullptr;
+  return g_ctx_current(&ctx) == CUDA_SUCCESS ? ctx : nullptr;
+}
 
 // Device address of the scratch on the current device.  Host code cannot use
 // the array's name as an address (it is a host-side stand-in), so the first
 // call on each device asks the runtime for it, with that device current, and
-// keeps the answer.
+// keeps the answer for that device's current context.
 cudaError_t scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_dev[dev] == nullptr) {
+  CUcontext ctx = current_context();
+  ScratchEntry& ent = g_scratch_dev[dev];
+  if (ent.ptr == nullptr || ctx == nullptr || ent.ctx != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_append_scratch);
+    e = cudaGetSymbolAddress(&p, g_append_scratch);  // makes the device's primary context current if needed
     if (e != cudaSuccess) return e;
-    g_scratch_dev[dev] = p;
+    ent.ctx = current_context();
+    ent.ptr = p;
   }
-  *out = g_scratch_dev[dev];
+  *out = ent.ptr;
   return cudaSuccess;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+namespace mlra {
+// Forgets every cached scratch address (mlra_shutdown calls this).
+void noalloc_forget_scratch() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (ScratchEntry& ent : g_scratch_dev) ent = ScratchEntry{};
+}
+}  // namespace mlra
 
 extern "C" MLRA_API mlra_status latent_append_noalloc(const mlra_dims* dims, int d_model, const void* h,
                                                       const void* W_DKV, const void* W_KR, const int32_t* pos,

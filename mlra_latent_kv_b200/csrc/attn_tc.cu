@@ -18,10 +18,13 @@
 //     (four with one branch per CTA, two with two).
 //   * MLA (one softmax over all 512 dims): CTA r computes the partial scores
 //     of its 256 latent dims and of its 32 of the 64 rope dims.  Exchange warps
-//     send each page's partial (rounded to fp16) to the peer through
-//     distributed shared memory as soon as QK^T has produced it; both CTAs add
-//     f16(own) + f16(peer's), so they hold the same bits and compute identical
-//     softmax weights.
+//     send each page's partial to the peer through distributed shared memory
+//     as soon as QK^T has produced it, as the row's maximum r over the page's
+//     tokens (fp32) and each score's offset from it, s - r, rounded to fp16.
+//     Both CTAs then form (r_0 + r_1) + (f16(s_0 - r_0) + f16(s_1 - r_1)):
+//     fp32 addition commutes, so they hold the same bits and compute identical
+//     softmax weights, and the rounding error of a score is 2^-11 of its
+//     distance below its row's page maximum, however large the logits.
 //   * MLRA with 2 or 4 branches: the branches of a CTA are wholly its own, so
 //     the CTAs of a worker never talk; each adds the full rope score to its
 //     branches.  MLRA-4 with more than 32 heads runs four CTAs per worker, one
@@ -123,13 +126,15 @@ struct Layout {
   static constexpr int kRopeQBytes = kExch ? kHq * 64 : kQSlotBytes;
   static constexpr int kRopeTileBytes = kExch ? 64 * 64 : kTileSlotBytes;
   static constexpr int kRopeRowBytes = kExch ? 64 : 128;
-  static constexpr int kXBytes = 64 * kHq * 2;   // one page of fp16 partial scores, kHq rows
+  static constexpr int kXBytes = 64 * kHq * 2;   // one page of fp16 score offsets, kHq rows
+  static constexpr int kXRBytes = kHq * 4;       // the fp32 row maxima they are offsets from
   static constexpr int kStageBytes = kLat * kTileSlotBytes + (kExch ? 0 : kRopeTileBytes);
   static constexpr int kQ = 0;
   static constexpr int kQRope = kLat * kQSlotBytes;
   static constexpr int kRope = kQRope + kRopeQBytes;  // MLA rope ring
   static constexpr int kX = kRope + (kExch ? 2 * kRopeTileBytes : 0);
-  static constexpr int kTile = (kX + (kExch ? kXBytes : 0) + 1023) / 1024 * 1024;
+  static constexpr int kXR = kX + (kExch ? kXBytes : 0);
+  static constexpr int kTile = (kXR + (kExch ? kXRBytes : 0) + 1023) / 1024 * 1024;
   static constexpr int kFixed = kTile + (int)sizeof(Bars) + 1024;  // + alignment slack
   static constexpr int kStages = (kCap - kFixed) / kStageBytes < kMaxStages ? (kCap - kFixed) / kStageBytes
                                                                               : kMaxStages;
@@ -234,6 +239,28 @@ __device__ __forceinline__ bool softmax_page(float (&s)[64], int valid, bool fir
   return rescale;
 }
 
+// Maximum of a row's scores over the page's first `valid` tokens (the exact
+// value does not depend on the order, so the exchange warp, which holds the
+// scores as two 32-column halves, and the softmax warp agree on it).
+__device__ __forceinline__ float row_max_valid(const uint32_t (&lo)[32], const uint32_t (&hi)[32], int valid) {
+  float m8[8];
+#pragma unroll
+  for (int n = 0; n < 64; ++n) {
+    const float v = n < valid ? __uint_as_float(n < 32 ? lo[n] : hi[n - 32]) : -INFINITY;
+    m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+  }
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+__device__ __forceinline__ float row_max_valid(const float (&s)[64], int valid) {
+  float m8[8];
+#pragma unroll
+  for (int n = 0; n < 64; ++n) {
+    const float v = n < valid ? s[n] : -INFINITY;
+    m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+  }
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
 template <bool kExch, int kBrPerCta, int kHq, int kCtas>
 __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCtas>())
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q_rope,
@@ -258,6 +285,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
   uint8_t* sTile = smem + L::kTile;
   uint8_t* sRope = smem + L::kRope;
   uint8_t* sX = smem + L::kX;
+  float* sXR = reinterpret_cast<float*>(smem + L::kXR);
   constexpr int kStages = L::kStages;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::kBars);
   volatile int* abort_flag = &bars->abort_flag;
@@ -296,7 +324,8 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
     mbar_init(smem_u32(&bars->o_free), 4 * kBrPerCta);
     // MLA: the peer's partial scores of page 0 are expected in phase 0 of x_full
     if (kExch)
-      for (int q = 0; q * 32 < a.H; ++q) mbar_expect_tx(smem_u32(&bars->x_full[q]), (uint32_t)min(32, a.H - q * 32) * 128u);
+      for (int q = 0; q * 32 < a.H; ++q)
+        mbar_expect_tx(smem_u32(&bars->x_full[q]), (uint32_t)min(32, a.H - q * 32) * (128u + 4u));
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -642,6 +671,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
     const uint32_t peer = rank ^ 1u;
     if (q4 * 32 < a.H) {
       const uint32_t dst = map_to_cta(smem_u32(sX), peer);
+      const uint32_t dst_r = map_to_cta(smem_u32(sXR), peer);
       const uint32_t bar = map_to_cta(smem_u32(&bars->x_full[q4]), peer);
       SegWalk walk(plan, a.B, maxL);
       uint32_t g = 0;
@@ -662,11 +692,13 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
           // (page g + kSB needs QK(g + kSB), hence P(g) written).
           if (lane == 0) mbar_arrive(smem_u32(&bars->xs_read[q4][g % kSB]));
           if (row == 0) MLRA_TRACE_EV(g, kEvXLoaded);
+          const int valid = min(kPage, walk.L - p * kPage);
+          const float r = row_max_valid(lo, hi, valid);
           uint32_t h[32];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            h[j] = pack_f16x2(__uint_as_float(lo[2 * j]), __uint_as_float(lo[2 * j + 1]));
-            h[16 + j] = pack_f16x2(__uint_as_float(hi[2 * j]), __uint_as_float(hi[2 * j + 1]));
+            h[j] = pack_f16x2(__uint_as_float(lo[2 * j]) - r, __uint_as_float(lo[2 * j + 1]) - r);
+            h[16 + j] = pack_f16x2(__uint_as_float(hi[2 * j]) - r, __uint_as_float(hi[2 * j + 1]) - r);
           }
           // single buffer: the peer warp must have read my page g-1
           if (g > 0 && !mbar_wait_warp<true>(smem_u32(&bars->x_empty[q4]), (g - 1) & 1, abort_flag, err,
@@ -680,6 +712,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
             for (int q = 0; q < 8; ++q)
               st_async_v4(dst + (uint32_t)((q * kHq + row) * 16), h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3],
                           bar);
+            st_async_b32(dst_r + (uint32_t)(row * 4), __float_as_uint(r), bar);
           }
           if (row == 0) MLRA_TRACE_EV(g, kEvSent);
         }
@@ -729,16 +762,21 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
           }
           if (row == 0) MLRA_TRACE_EV(g, kEvRecv);
           if (real) {
+            // s = (r_own + r_peer) + (f16(s_own - r_own) + f16(s_peer - r_peer)); each sum has the
+            // same operands on both CTAs, in the other order, so both get the same bits
+            const float r_own = row_max_valid(cur, valid);
+            const float r_sum = r_own + sXR[row];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const uint4 v = *reinterpret_cast<const uint4*>(sX + (q * kHq + row) * 16);
               const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const float2 mine = unpack_f16x2(pack_f16x2(cur[8 * q + 2 * j], cur[8 * q + 2 * j + 1]));
+                const float2 mine =
+                    unpack_f16x2(pack_f16x2(cur[8 * q + 2 * j] - r_own, cur[8 * q + 2 * j + 1] - r_own));
                 const float2 theirs = unpack_f16x2(w[j]);
-                cur[8 * q + 2 * j] = mine.x + theirs.x;
-                cur[8 * q + 2 * j + 1] = mine.y + theirs.y;
+                cur[8 * q + 2 * j] = r_sum + (mine.x + theirs.x);
+                cur[8 * q + 2 * j + 1] = r_sum + (mine.y + theirs.y);
               }
             }
           }
@@ -746,7 +784,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
           // page g consumed: arm the next phase, then let the peer refill the buffer
           __syncwarp();
           if (lane == 0) {
-            mbar_expect_tx(smem_u32(&bars->x_full[q4]), (uint32_t)q_rows * 128u);
+            mbar_expect_tx(smem_u32(&bars->x_full[q4]), (uint32_t)q_rows * (128u + 4u));
             mbar_arrive_cluster(map_to_cta(smem_u32(&bars->x_empty[q4]), peer));
           }
         }
@@ -908,6 +946,17 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
     default: return cudaErrorInvalidValue;
   }
 #undef MLRA_LAUNCH
+}
+
+const char* tc_variant_name(int H, int n_branch) {
+  const bool small = H <= 32;
+  switch (n_branch) {
+    case 1: return small ? "attend_tc_kernel<mla, cta pair, 32 query rows>" : "attend_tc_kernel<mla, cta pair>";
+    case 2: return small ? "attend_tc_kernel<mlra-2, cta pair, 32 query rows>" : "attend_tc_kernel<mlra-2, cta pair>";
+    case 4: return small ? "attend_tc_kernel<mlra-4, cta pair, 32 query rows>"
+                         : "attend_tc_kernel<mlra-4, four ctas, two per sm>";
+    default: return "none";
+  }
 }
 
 void tc_shutdown() { host_cache_clear(); }

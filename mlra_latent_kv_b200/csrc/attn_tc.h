@@ -21,6 +21,9 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
                              const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                              cudaStream_t st, bool pdl);
 
+// Name of the attention kernel variant launch_attend_tc picks for this shape.
+const char* tc_variant_name(int H, int n_branch);
+
 // Frees the host-side tensor-map cache.
 void tc_shutdown();
 

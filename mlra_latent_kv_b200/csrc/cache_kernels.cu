@@ -162,7 +162,8 @@ __global__ void append_finalize_kernel(const float* __restrict__ part, const int
     report_error(err, kErrDeviceCheck, b, p);
     return;
   }
-  const int pg = page_of(page_table, a.maxp, a.num_pages, b, p, err);
+  const int pg = page_for_write(page_table, a.maxp, a.num_pages, b, p, err);
+  if (pg < 0) return;  // reported; nothing is written for this sequence
   const size_t slot = (size_t)pg * kPage + (p % kPage);
   if (j < a.d_c) {
     lat[slot * a.d_c + j] = from_f<T>(x0);
@@ -234,7 +235,8 @@ __global__ void store_kernel(const T* __restrict__ c_kv, const T* __restrict__ k
       report_error(err, kErrDeviceCheck, i, p);
       continue;
     }
-    const int pg = page_of(page_table, a.maxp, a.num_pages, b, p, err);
+    const int pg = page_for_write(page_table, a.maxp, a.num_pages, b, p, err);
+    if (pg < 0) continue;  // reported; this token is not written
     const size_t slot = (size_t)pg * kPage + (p % kPage);
     if (k < lchunks) {
       const uint4 v = *reinterpret_cast<const uint4*>(c_kv + (size_t)i * a.d_c + (size_t)k * kPer16);

@@ -38,14 +38,28 @@ __device__ __forceinline__ void report_error(int* rec, int code, int a, int b) {
   }
 }
 
-// Page id of token t of sequence b; an id outside [0, num_pages) is reported
-// and replaced by page 0 so that no access leaves the pool.
+// Page id of token t of sequence b for a READ; an id outside [0, num_pages)
+// is reported and replaced by page 0, so that no read leaves the pool (the
+// call's result is void, and mlra_check_status says so).
 __device__ __forceinline__ int page_of(const int* page_table, int maxp, int num_pages, int b, int t,
                                        int* err) {
   int pg = __ldg(page_table + (size_t)b * maxp + t / kPage);
   if (pg < 0 || pg >= num_pages) {
     report_error(err, kErrDeviceCheck, b, t);
     pg = 0;
+  }
+  return pg;
+}
+
+// Page id of token t of sequence b for a WRITE; an id outside [0, num_pages)
+// is reported and -1 returned: the caller skips the store, because page 0 (or
+// any other stand-in) belongs to some other live sequence.
+__device__ __forceinline__ int page_for_write(const int* page_table, int maxp, int num_pages, int b, int t,
+                                              int* err) {
+  const int pg = __ldg(page_table + (size_t)b * maxp + t / kPage);
+  if (pg < 0 || pg >= num_pages) {
+    report_error(err, kErrDeviceCheck, b, t);
+    return -1;
   }
   return pg;
 }

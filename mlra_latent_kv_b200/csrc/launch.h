@@ -58,6 +58,8 @@ cudaError_t launch_store(int dtype, const void* c_kv, const void* k_rope, const 
 #include "../../include/mlra.h"
 
 namespace mlra {
+// defined in append_noalloc.cu
+void noalloc_forget_scratch();
 // defined in mlra_api.cu
 mlra_status internal_check_dims(const mlra_dims* d);
 mlra_status internal_fail(mlra_status st, const char* msg);

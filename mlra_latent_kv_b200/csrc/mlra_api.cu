@@ -221,6 +221,25 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
 
 extern "C" {
 
+mlra_status mlra_describe_plan(const mlra_dims* dims, char* buf, size_t buf_len) {
+  if (!buf || buf_len == 0) return fail(MLRA_ERR_INVALID_ARG, "buf is NULL or empty");
+  DecodePlan p;
+  mlra_status st = make_plan(dims, &p);
+  if (st != MLRA_OK) return st;
+  const mlra_dims* d = dims;
+  const bool tc_absorb = p.tc && absorb_tc_supported(d->dtype, d->B, d->d_h, d->d_c);
+  const bool tc_upproj = p.tc && upproj_tc_supported(d->dtype, d->B, d->d_c, d->d_v, p.G, d->n_branch);
+  const char* family = !p.tc ? "cuda-core" : (tc_absorb && tc_upproj ? "tcgen05" : "tcgen05+cuda-core");
+  const int n = snprintf(buf, buf_len,
+                         "family=%s;splits=%d;kernels=%d;absorb=%s;attention=%s;combine=%s;upproj=%s", family, p.G,
+                         2 + (tc_upproj ? 1 : 2), tc_absorb ? "absorb_tc_kernel" : "absorb_kernel",
+                         p.tc ? tc_variant_name(d->H, d->n_branch) : "attend_simt_kernel",
+                         tc_upproj ? "fused into combine_upproj_tc_kernel" : "combine_kernel",
+                         tc_upproj ? "combine_upproj_tc_kernel" : "upproj_kernel");
+  if (n < 0 || (size_t)n >= buf_len) return fail(MLRA_ERR_INVALID_ARG, "buf too small (%d bytes needed)", n + 1);
+  return MLRA_OK;
+}
+
 size_t mlra_workspace_bytes(const mlra_dims* dims) {
   DecodePlan p;
   if (make_plan(dims, &p) != MLRA_OK) return 0;
@@ -394,7 +413,10 @@ mlra_status mlra_check_status(void* workspace, cudaStream_t stream) {
 
 const char* mlra_last_error(void) { return g_err.c_str(); }
 
-void mlra_shutdown(void) { tc_shutdown(); }
+void mlra_shutdown(void) {
+  tc_shutdown();
+  noalloc_forget_scratch();
+}
 
 int mlra_version(void) { return 1; }
 

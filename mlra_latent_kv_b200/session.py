@@ -115,14 +115,10 @@ class DecodeSession:
             abi.check_status(self.app_ws)
 
     def kernels_per_step(self) -> int:
-        """Kernels one step launches: append (2, when it appends), absorption,
-        attention, and combine + up-projection (one fused tcgen05 kernel, or two
-        CUDA-core kernels), following the library's kernel choice."""
-        w = self.w
-        tc = (self.dims.kernel != 1 and w.dtype == "bf16" and w.d_c == 512 and w.d_r == 64 and w.H <= 128
-              and w.n_branch in (1, 2, 4))
-        G = self.dims.num_splits or torch.cuda.get_device_properties(self.device).multi_processor_count // 2
-        bp = 16 if w.B <= 16 else (w.B + 15) // 16 * 16
-        smem = 1024 + 2 * w.d_c * 128 + (w.d_c // 64) * bp * 128 + 3 * (G + w.B) * w.n_branch * 4 + 2 * w.B * 4 + G * 4
-        fused = tc and w.B <= 96 and w.d_v % 128 == 0 and smem <= 232448
-        return (2 if self.appends else 0) + 2 + (1 if fused else 2)
+        """Kernels one step launches: append (2, when it appends) plus the
+        decode call's own launches, as the library plans them."""
+        return (2 if self.appends else 0) + abi.describe_plan(self.dims)["kernels"]
+
+    def plan(self) -> dict:
+        """The decode call's kernel plan (family and per-stage kernel names)."""
+        return abi.describe_plan(self.dims)

@@ -145,3 +145,39 @@ def test_append_and_store_validation(L):
 def test_selftest_validation(L):
     assert L.mlra_selftest_wait_timeout(None, 1000, None) == 1
     assert L.mlra_selftest_wait_timeout(1 << 20, 0, None) == 1
+
+
+def _workload_dims(w, num_splits=74):
+    from mlra_latent_kv_b200 import synth  # noqa: F401
+    return abi.make_dims(B=w.B, H=w.H, d_h=w.d_h, d_v=w.d_v, d_c=w.d_c, d_r=w.d_r, max_pages_per_seq=8,
+                         num_pages=32, n_branch=w.n_branch, branch_scale=w.branch_scale, dtype=w.dtype,
+                         num_splits=num_splits)
+
+
+def test_every_bf16_workload_plans_the_tcgen05_family(L):
+    """Kernel AUTO puts every bf16 workload of the decode study on the tcgen05
+    kernels (no silent CUDA-core stage); the fp32 tiny workload runs on the
+    CUDA-core kernels, which are the ones that take fp32."""
+    from mlra_latent_kv_b200 import synth
+    for w in synth.WORKLOADS:
+        plan = abi.describe_plan(_workload_dims(w))
+        if w.dtype == "bf16":
+            assert plan["family"] == "tcgen05", (w.name, plan)
+            assert plan["attention"].startswith("attend_tc_kernel"), (w.name, plan)
+            assert plan["kernels"] == 3, (w.name, plan)
+        else:
+            assert plan["family"] == "cuda-core", (w.name, plan)
+            assert plan["kernels"] == 4, (w.name, plan)
+        assert plan["splits"] == 74
+
+
+def test_describe_plan_follows_the_kernel_switch(L):
+    from mlra_latent_kv_b200 import synth
+    w = synth.workload("mlra4")
+    d = _workload_dims(w)
+    d.kernel = 1
+    assert abi.describe_plan(d)["family"] == "cuda-core"
+    d.kernel = 2
+    assert abi.describe_plan(d)["attention"] == "attend_tc_kernel<mlra-4, four ctas, two per sm>"
+    buf = ctypes.create_string_buffer(8)
+    assert L.mlra_describe_plan(ctypes.byref(d), buf, len(buf)) == 1  # MLRA_ERR_INVALID_ARG

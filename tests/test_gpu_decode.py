@@ -142,6 +142,86 @@ def test_dominant_key_is_selected(kernel):
     assert err <= tol
 
 
+def _scale_with_exact_log2(target=0.125):
+    """A softmax scale whose fp32 product with log2(e) (the kernels' base-2
+    logit scale) is exactly ``target``, so the absorbed query loses nothing."""
+    c = np.float32(1.4426950408889634)
+    s = np.float32(target / 1.4426950408889634)
+    for _ in range(8):
+        p = np.float32(s * c)
+        if p == np.float32(target):
+            return float(s)
+        s = np.nextafter(s, np.float32(np.inf if p < target else -np.inf), dtype=np.float32)
+    raise AssertionError("no fp32 scale found")
+
+
+def _peaked_inputs(w, peak_log2, n_plant, seed):
+    """Peaked attention with many near-ties, built so that every rounding on the
+    GPU path except the scores' own arithmetic is exact: W_UK rows are one-hot
+    (q_lat is q_nope placed on 128 latent dims, 64 in each half of the 512),
+    q_nope entries are +-(1 + k 2^-7) (bf16-exact), latents are small
+    integers, the base-2 logit scale is 1/8 exactly and there is no rope
+    term.  So every QK^T partial is exact in fp32, and a score's error can
+    only come from how the two halves' partials are combined.  n_plant tokens
+    per sequence, spread over its pages (hence over split workers), carry
+    logits near ``peak_log2`` (log2 units) within about +-0.6 of each other;
+    the other tokens sit near 0.  W_UV is zero on the score dims, so the
+    planted tokens' values differ (from their other 384 latent dims)."""
+    inp = synth.make_inputs(w)
+    rng = np.random.default_rng(seed)
+    sel = np.concatenate([np.arange(0, 256, 4), 256 + np.arange(0, 256, 4)])
+    Wk = np.zeros((w.d_h, w.d_c))
+    Wk[np.arange(w.d_h), sel] = 1.0
+    inp["W_UK"] = torch.from_numpy(np.tile(Wk, (w.H, 1, 1))).to(torch.bfloat16)
+    u = rng.choice([-1.0, 1.0], w.d_h)
+    q = u * (1.0 + rng.integers(0, 128, (w.B, w.H, w.d_h)) * 2.0 ** -7)
+    inp["q_nope"] = torch.from_numpy(q).to(torch.bfloat16)
+    assert np.array_equal(inp["q_nope"].double().numpy(), q)
+    inp["q_rope"].zero_()
+    T = inp["c_kv"].shape[0]
+    C = rng.integers(-2, 3, (T, w.d_c)).astype(np.float64)
+    alpha = int(round(peak_log2 / (0.125 * 1.5 * w.d_h)))   # planted logit ~ alpha * sum|q| / 8
+    for b in range(w.B):
+        rows = np.where(inp["tok_seq"].numpy() == b)[0]
+        L = len(rows)
+        for t in np.linspace(3, L - 3, n_plant).astype(int) + rng.integers(-2, 3, n_plant):
+            c = C[rows[t]]
+            c[sel] = alpha * u
+            flip = rng.choice(sel, rng.integers(0, 4), replace=False)
+            c[flip] += rng.choice([-1.0, 1.0], len(flip))
+    inp["c_kv"] = torch.from_numpy(C).to(torch.bfloat16)
+    assert np.array_equal(inp["c_kv"].double().numpy(), C)
+    Wv = inp["W_UV"].clone()
+    Wv[:, sel, :] = 0
+    inp["W_UV"] = Wv
+    return inp
+
+
+@pytest.mark.parametrize("G", [0, 3])
+@pytest.mark.parametrize("peak", [120.0, 240.0])
+@pytest.mark.parametrize("H", [128, 32])
+def test_peaked_attention_near_ties(H, peak, G):
+    """Logits of 100-300 log2 units with 8 near-tied keys per sequence, in
+    different pages and split workers: the combination of the two CTAs'
+    partial scores must keep each score accurate to a small fraction of a
+    log2 unit, or the near-tied weights (and so the output) move."""
+    w = synth.workload("dsv2_contiguous").with_(B=3, H=H, seq_len=1500, paged=True, seed=17)
+    inp = _peaked_inputs(w, peak, 8, seed=170 + H)
+    ss = _scale_with_exact_log2()
+    s = DecodeSession(w, inp, num_splits=G)
+    s.dims.softmax_scale = ss
+    out = s.step().clone()
+    torch.cuda.synchronize()
+    s.check()
+    oi = oracle_inputs(w, inp)
+    oi["softmax_scale"] = ss
+    ref = oracle.decode(oi)
+    top = max(float(np.max(v)) for v in ref.values())
+    assert top > 0.1   # the values are not all zero (W_UV keeps 384 latent dims)
+    err, tol = compare(out, ref)
+    assert err <= tol, f"H={H} peak={peak} G={G}: {err:.3e} > {tol:.3e} (rel l2 {rel_l2(out, ref):.2e})"
+
+
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_device_check_bad_page_id(kernel):
     w = synth.workload("dsv2_contiguous").with_(B=2, seq_len=100)
