@@ -11,8 +11,13 @@ launching stream and the job time is the max over ranks.  With N > 1 (one
 process per GPU, torchrun) every rank decodes its own batch: weak scaling, no
 data-path collective.
 
+The default workload is the paged variable-length batch at H = 32 (the
+largest single-GPU workload); the same run also times the split-KV attention
+kernel of the MLRA-4 workload (reported under roofline_by_workload).
+
 --impl reference times the fp64 CPU oracle on the host cores instead (a
-bounded sample of (sequence, head) pairs per step, extrapolated to the step).
+bounded sample of (sequence, head) pairs per step, extrapolated to the step),
+with the same sampler as the cpu_baseline leg.
 """
 from __future__ import annotations
 
@@ -24,6 +29,7 @@ import statistics
 import sys
 import threading
 import time
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -35,7 +41,8 @@ from mlra_latent_kv_b200 import dist as mdist  # noqa: E402
 from mlra_latent_kv_b200 import synth  # noqa: E402
 
 METRIC = "latent decode attention µs/step, achieved HBM GB/s and % of 1×B200 roofline"
-DEFAULT_WORKLOAD = "dsv2_contiguous"
+DEFAULT_WORKLOAD = "paged_varlen_h32"
+COMPANION_WORKLOADS = ("mlra4",)   # attention roofline also reported for these (1-GPU runs)
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -144,47 +151,69 @@ def captured_traffic(workload: str):
 # oracle timing (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
 
-def oracle_threads() -> int:
+def host_cores() -> int:
+    """Host cores this process may run on (the oracle's thread pool size)."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:  # noqa: BLE001
-        return 1
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
 
 
-def time_oracle_pairs(w, inp, pairs) -> float:
-    import oracle
-    from oracle.inputs import oracle_inputs
-    oi = oracle_inputs(w, inp)
-    t0 = time.perf_counter()
-    oracle.decode(oi, pairs)
-    return time.perf_counter() - t0
+class OracleSampler:
+    """Times the fp64 oracle, as it stands, on random (sequence, head) pairs of
+    one workload step: the pairs are split into chunks that a pool of one
+    thread per host core runs through ``oracle.decode`` (its BLAS calls held
+    to one thread each, so the pool is the parallelism).  The wall time of a
+    sample scales to a full step by B*H / pairs."""
 
+    def __init__(self, w, inp):
+        import oracle
+        from oracle.inputs import oracle_inputs
+        self._decode = oracle.decode
+        self.w = w
+        self.oi = oracle_inputs(w, inp)
+        self.cores = host_cores()
+        self.total = w.B * w.H
 
-def pick_pairs(w, n, seed=0):
-    rng = np.random.default_rng(12345 + seed)
-    bs = rng.integers(0, w.B, n)
-    hs = rng.integers(0, w.H, n)
-    return [(int(b), int(h)) for b, h in zip(bs, hs)]
+    def pairs(self, n, seed):
+        rng = np.random.default_rng(12345 + seed)
+        idx = rng.choice(self.total, size=n, replace=False)
+        return [(int(i) // self.w.H, int(i) % self.w.H) for i in idx]
+
+    def time(self, pairs) -> float:
+        from threadpoolctl import threadpool_limits
+        n_chunks = min(len(pairs), 4 * self.cores)
+        chunks = [pairs[i::n_chunks] for i in range(n_chunks)]
+        with threadpool_limits(1), ThreadPoolExecutor(self.cores) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(lambda c: self._decode(self.oi, c), chunks))
+            return time.perf_counter() - t0
+
+    def grow(self, budget_s, seed=1):
+        """Sample size whose timing takes at least half of budget_s (or the whole
+        step); returns (pairs, seconds)."""
+        n = min(self.total, 4 * self.cores)
+        t = self.time(self.pairs(n, seed))
+        while t < 0.5 * budget_s and n < self.total:
+            n = min(self.total, max(n + 1, int(n * budget_s / max(t, 1e-3))))
+            t = self.time(self.pairs(n, seed))
+        return n, t
+
+    def sample_text(self, n):
+        return (f"{n} random (sequence, head) pairs of the {self.w.name} step per timing, run by "
+                f"{self.cores} threads (one per host core, BLAS single-threaded), scaled by "
+                f"{self.total}/{n} to one step")
 
 
 def cpu_baseline(w, inp, budget_s: float = 15.0) -> dict:
     """The oracle (as it stands) on a bounded sample of (b, h) pairs, scaled to a full step."""
-    time_oracle_pairs(w, inp, pick_pairs(w, 8, seed=6))  # warm (first-touch costs are not the oracle's rate)
-    # grow the sample until it takes about half the budget or covers the whole step (the
-    # oracle's per-pair cost falls with the sample size, so one small calibration overshoots)
-    n = min(w.B * w.H, 64)
-    t = time_oracle_pairs(w, inp, pick_pairs(w, n, seed=1))
-    while t < 0.5 * budget_s and n < w.B * w.H:
-        n = min(w.B * w.H, max(n + 1, int(n * budget_s / max(t, 1e-3))))
-        t = time_oracle_pairs(w, inp, pick_pairs(w, n, seed=1))
-    per_pair = t / n
-    step_s = per_pair * w.B * w.H
+    smp = OracleSampler(w, inp)
+    smp.time(smp.pairs(min(smp.total, smp.cores), seed=6))  # first-touch costs are not the oracle's rate
+    n, t = smp.grow(budget_s)
+    step_s = t * smp.total / n
     sb = step_bytes(w, inp)
-    return {"value": sb["total"] / step_s / 1e9, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{n} random (sequence, head) pairs of the {w.name} step in {t:.1f} s, "
-                      f"scaled by {w.B * w.H}/{n} to one step ({step_s:.1f} s/step)",
+    return {"value": sb["total"] / step_s / 1e9, "unit": "GB/s", "cores": smp.cores, "kind": "oracle",
+            "sample": smp.sample_text(n) + f" ({t:.1f} s for the sample, {step_s:.1f} s/step)",
             "s_per_step": step_s}
 
 
@@ -194,25 +223,25 @@ def run_reference(args, w):
         return 0
     inp = synth.make_inputs(w)
     sb = step_bytes(w, inp)
-    t1 = time_oracle_pairs(w, inp, pick_pairs(w, 1))
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    per_step = max(1, min(w.B * w.H, int(budget / max(t1, 1e-6))))
+    smp = OracleSampler(w, inp)
+    # the cpu_baseline leg's sampler and growth rule, with a per-step budget that keeps the
+    # whole --steps/--warmup run to a few minutes
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    n, _ = smp.grow(budget, seed=99)
     for i in range(args.warmup):
-        time_oracle_pairs(w, inp, pick_pairs(w, per_step, seed=100 + i))
+        smp.time(smp.pairs(n, seed=100 + i))
     tot = 0.0
     for i in range(args.steps):
-        tot += time_oracle_pairs(w, inp, pick_pairs(w, per_step, seed=1000 + i))
-    step_s = tot / (args.steps * per_step) * w.B * w.H
+        tot += smp.time(smp.pairs(n, seed=1000 + i))
+    step_s = tot / args.steps * smp.total / n
     value = sb["total"] / step_s / 1e9
-    cores = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, inp, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{per_step} random (sequence, head) pairs per step, scaled by "
-                                   f"{w.B * w.H}/{per_step} to the full step"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": smp.cores, "kind": "oracle",
+                         "sample": smp.sample_text(n) + "; one fresh sample per step"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -234,6 +263,70 @@ def config_of(w, inp, n):
 # our arm
 # ---------------------------------------------------------------------------
 
+def roofline_of(sb, attn_us, peaks, src) -> dict:
+    """Roofline of the split-KV attention kernel from its event-timed duration:
+    the bound is whichever of cache bytes / HBM peak and attention flops /
+    bf16 tensor peak is longer (burst peaks: the kernel is timed on its own,
+    well under a second); achieved, peak and frac are reported for that bound,
+    the other pipe's figures beside them."""
+    hbm = float(peaks["hbm_gbs"])
+    tc = float(peaks["bf16_tflops"])
+    attn_s = attn_us * 1e-6
+    t_hbm = sb["cache"] / (hbm * 1e9)
+    t_tc = sb["attn_flops"] / (tc * 1e12)
+    gbs = sb["cache"] / attn_s / 1e9
+    tfs = sb["attn_flops"] / attn_s / 1e12
+    hbm_bound = t_hbm >= t_tc
+    note = "of measured" if src == "measured" else "of fallback"
+    return {"kernel": "split-KV latent attention", "bound": "hbm" if hbm_bound else "tensor",
+            "achieved": gbs if hbm_bound else tfs, "peak": hbm if hbm_bound else tc,
+            "unit": "GB/s" if hbm_bound else "TFLOP/s", "frac": (gbs / hbm) if hbm_bound else (tfs / tc),
+            "peak_source": f"{note} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops burst)",
+            "algorithmic_bytes_per_launch": sb["cache"], "algorithmic_flops_per_launch": sb["attn_flops"],
+            "attn_us": attn_us, "hbm_gbs": gbs, "hbm_frac": gbs / hbm, "tensor_tflops": tfs, "tensor_frac": tfs / tc,
+            "tensor_peak_tflops": tc, "hbm_peak_gbs": hbm,
+            "roofline_us": max(t_hbm, t_tc) * 1e6, "frac_of_roofline_time": max(t_hbm, t_tc) / attn_s}
+
+
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def staged_timing(sess, stream, flush, K, W, graph=True):
+    """Per-stage device times (µs, mean over K steps) of one decode step with
+    events recorded between its kernels (which serialises them), L2 flushed
+    before every step."""
+    stage = _events(5)
+    for e in stage:  # materialise the raw events before handing them to the library
+        e.record(stream)
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            sess.step(events=stage)
+    for _ in range(W):
+        flush.fill_(3)
+        g.replay() if g else sess.step(events=stage)
+    torch.cuda.synchronize()
+    acc = {"absorb": 0.0, "attention": 0.0, "combine": 0.0, "upproj_incl_fused_combine": 0.0}
+    if sess.appends:
+        acc["append"] = 0.0
+    starts = _events(K)
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        g.replay() if g else sess.step(events=stage)
+        stage[4].synchronize()
+        for name, a, b in (("absorb", 0, 1), ("attention", 1, 2), ("combine", 2, 3),
+                           ("upproj_incl_fused_combine", 3, 4)):
+            acc[name] += stage[a].elapsed_time(stage[b])
+        if sess.appends:
+            acc["append"] += starts[i].elapsed_time(stage[0])
+    torch.cuda.synchronize()
+    del g
+    return {k: v / K * 1e3 for k, v in acc.items()}
+
+
 def run_ours(args, w):
     from mlra_latent_kv_b200.session import DecodeSession
     rank, ws, local = mdist.world()
@@ -246,75 +339,45 @@ def run_ours(args, w):
     sb = step_bytes(wr, inp)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def mk(n):
-        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-
     K, W = args.steps, args.warmup
-    starts, ends = mk(K), mk(K)
-    stage = mk(5)
-    for e in stage:  # materialise the raw events before handing them to the library
-        e.record(stream)
+    starts, ends = _events(K), _events(K)
     for _ in range(W):
         flush.fill_(1)
         sess.step()
     torch.cuda.synchronize(dev)
     sess.check()
-    # One decode step captured as a CUDA graph, replayed once per timed step.
-    # The headline pass replays the plain step (its kernels chained by
-    # programmatic dependent launches); a second timed pass replays a step with
-    # the stage events recorded between the kernels (which also serialises
-    # them) for the per-kernel times and the attention roofline.
-    graphs = {}
+    # The headline pass replays one decode step captured as a CUDA graph (its
+    # kernels chained by programmatic dependent launches); a second timed pass
+    # (staged_timing) records events between the kernels for the per-kernel
+    # times and the attention roofline.
+    graph = None
     if not args.no_graph:
-        for name, evs in (("plain", None), ("staged", stage)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                sess.step(events=evs)
-            for _ in range(W):
-                flush.fill_(1)
-                g.replay()
-            graphs[name] = g
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            sess.step()
+        for _ in range(W):
+            flush.fill_(1)
+            graph.replay()
         torch.cuda.synchronize(dev)
 
-    def one_step(staged: bool):
-        if graphs:
-            graphs["staged" if staged else "plain"].replay()
-        else:
-            sess.step(events=stage if staged else None)
-
-    stage_acc = {"absorb": 0.0, "attention": 0.0, "combine": 0.0, "upproj_incl_fused_combine": 0.0}
-    if sess.appends:
-        stage_acc["append"] = 0.0
     mdist.barrier(dev)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(K):
             flush.fill_(i & 0xFF)
             starts[i].record(stream)
-            one_step(False)
+            graph.replay() if graph is not None else sess.step()
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
         mdist.barrier(dev)
-        s_starts = mk(K)
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            s_starts[i].record(stream)
-            one_step(True)
-            stage[4].synchronize()
-            for name, a, b in (("absorb", 0, 1), ("attention", 1, 2), ("combine", 2, 3),
-                               ("upproj_incl_fused_combine", 3, 4)):
-                stage_acc[name] += stage[a].elapsed_time(stage[b])
-            if sess.appends:
-                stage_acc["append"] += s_starts[i].elapsed_time(stage[0])
-        torch.cuda.synchronize(dev)
+        stage_us = staged_timing(sess, stream, flush, K, W, graph=not args.no_graph)
     mdist.barrier(dev)
     torch.cuda.synchronize(dev)
     sess.check()
+    del graph
 
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
-    stage_ms = {k: v / K for k, v in stage_acc.items()}
     max_total_ms = mdist.max_over_ranks(total_ms, dev)
     value = mdist.throughput(sb["total"] * K, ws, max_total_ms / 1e3) / 1e9
 
@@ -337,7 +400,16 @@ def run_ours(args, w):
             sess.append()
         sess.decode_host(host["q_nope"], host["q_rope"], host["q_pos"], host["seq_lens"], out_host)
 
-    e_s, e_e = mk(K), mk(K)
+    # the same host<->device copies alone, for the split of the e2e step
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in list(host.items()) + list(app_host.items())}
+    dev_out = torch.empty(sess.out.shape, dtype=sess.out.dtype, device=dev)
+
+    def copies_only():
+        for k, v in list(host.items()) + list(app_host.items()):
+            dev_in[k].copy_(v, non_blocking=True)
+        out_host.copy_(dev_out, non_blocking=True)
+
+    e_s, e_e = _events(K), _events(K)
     for _ in range(W):
         flush.fill_(2)
         e2e_step()
@@ -352,44 +424,67 @@ def run_ours(args, w):
     sess.check()
     e2e_ms = mdist.max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)), dev)
     e2e_value = mdist.throughput(sb["total"] * K, ws, e2e_ms / 1e3) / 1e9
+    c_s, c_e = _events(K), _events(K)
+    for i in range(K):
+        c_s[i].record(stream)
+        copies_only()
+        c_e[i].record(stream)
+    torch.cuda.synchronize(dev)
+    copy_ms = sum(a.elapsed_time(b) for a, b in zip(c_s, c_e)) / K
 
     peaks, src = load_peaks()
-    attn_s = stage_ms["attention"] / 1e3
-    hbm_peak = float(peaks["hbm_gbs"])
-    achieved = sb["cache"] / attn_s / 1e9
-    tflops = sb["attn_flops"] / attn_s / 1e12
-    tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    roofline_t = max(sb["cache"] / (hbm_peak * 1e9), sb["attn_flops"] / (float(peaks["bf16_tflops"]) * 1e12))
-    traffic = captured_traffic(w.name)
+    roof = roofline_of(sb, stage_us["attention"], peaks, src)
+    roof["traffic"] = captured_traffic(w.name)
+    plan = sess.plan()
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W,
         "ms_per_step": max_total_ms / K, "us_per_step": max_total_ms / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded per workload, shapes of the workload configuration)",
         "config": config_of(w, inp, ws),
-        "stage_us": {k: v * 1e3 for k, v in stage_ms.items()},
-        "roofline": {"kernel": "split-KV latent attention", "bound": "hbm", "achieved": achieved,
-                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
-                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
-                     "algorithmic_bytes_per_launch": sb["cache"], "attn_us": stage_ms["attention"] * 1e3,
-                     "tensor_tflops": tflops, "tensor_peak_tflops": tensor_peak,
-                     "roofline_us": roofline_t * 1e6, "frac_of_roofline_time": roofline_t / attn_s},
+        "stage_us": stage_us,
+        "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "mlra_decode_host (host buffers; copies inside the timed region)",
-                "ms_per_step": e2e_ms / K},
+                "ms_per_step": e2e_ms / K,
+                "copies_alone_ms_per_step": copy_ms},
         "gpu_launches": K * sess.kernels_per_step(),
+        "kernels": plan,
         "timed_as": ("eager API calls" if args.no_graph else "CUDA graph replay of one decode step per timed step")
                     + "; stage_us and roofline from a second timed pass with events between the kernels",
         "clocks": clk.summary(),
         "step_bytes": sb,
     }
+    del sess
+    torch.cuda.empty_cache()
+
+    # the split-KV attention of the other target workloads, timed the same way (1-GPU runs)
+    if ws == 1 and not args.no_companions:
+        by = {}
+        for name in COMPANION_WORKLOADS:
+            if name == w.name:
+                continue
+            cw = synth.workload(name)
+            cinp = synth.make_inputs(cw)
+            cs = DecodeSession(cw, cinp, device=dev, kernel=args.kernel)
+            with ClockSampler(local) as cclk:
+                cst = staged_timing(cs, stream, flush, min(K, 50), W, graph=not args.no_graph)
+            cs.check()
+            csb = step_bytes(cw, cinp)
+            r = roofline_of(csb, cst["attention"], peaks, src)
+            r["traffic"] = captured_traffic(name)
+            by[name] = {"roofline": r, "stage_us": cst, "kernels": cs.plan(), "clocks": cclk.summary(),
+                        "config": config_of(cw, cinp, ws)}
+            del cs
+            torch.cuda.empty_cache()
+        line["roofline_by_workload"] = by
+
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wr, inp)
     elif rank == 0:
         line["cpu_baseline"] = None
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del sess
     mdist.shutdown()
     return 0
 
@@ -403,6 +498,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-companions", action="store_true",
+                    help="skip the attention timing of the other target workloads")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of as a graph")
     args = ap.parse_args()
     if args.warmup < 3:

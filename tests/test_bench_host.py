@@ -60,3 +60,40 @@ def test_source_digest_follows_every_attention_source(tmp_path, monkeypatch):
         assert bench.source_digest() != base, f"{name} is not covered by the digest"
         p.write_bytes(orig)
     assert bench.source_digest() == base
+
+
+def _peaks():
+    return {"hbm_gbs": 6545.3, "bf16_tflops": 1618.5, "bf16_tflops_sustained": 1374.0}
+
+
+def test_roofline_bound_follows_the_arithmetic():
+    """HBM-bound at H = 32 (60 flop/B); at H = 128 the MLRA-4 step is HBM-bound
+    by a hair (92.3 us of bytes against 90.2 us of flops at these peaks); a
+    hypothetical 4x-flop kernel flips to the tensor bound."""
+    for name, bound in (("paged_varlen_h32", "hbm"), ("mlra4", "hbm")):
+        w = synth.workload(name)
+        inp = {"attn_lens": torch.full((w.B,), w.seq_len or 16000, dtype=torch.int32)}
+        sb = bench.step_bytes(w, inp)
+        r = bench.roofline_of(sb, 200.0, _peaks(), "measured")
+        assert r["bound"] == bound and r["unit"] == "GB/s"
+        assert abs(r["frac"] - sb["cache"] / 200e-6 / 1e9 / 6545.3) < 1e-12
+        assert r["tensor_peak_tflops"] == 1618.5          # the burst peak, the one the bound used
+        t = max(sb["cache"] / 6545.3e9, sb["attn_flops"] / 1618.5e12)
+        assert abs(r["roofline_us"] - t * 1e6) < 1e-6
+    sb = dict(cache=1e9, attn_flops=4 * 247 * 1e9 * 1.1)
+    r = bench.roofline_of(sb, 1000.0, _peaks(), "measured")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1618.5
+    assert abs(r["frac"] - sb["attn_flops"] / 1e-3 / 1e12 / 1618.5) < 1e-12
+
+
+def test_oracle_sampler_grows_and_scales_to_the_step():
+    w = synth.workload("dsv2_contiguous").with_(B=3, H=4, seq_len=200)
+    inp = synth.make_inputs(w)
+    smp = bench.OracleSampler(w, inp)
+    assert smp.cores == bench.host_cores() >= 1
+    p = smp.pairs(5, seed=1)
+    assert len(set(p)) == 5 and all(0 <= b < 3 and 0 <= h < 4 for b, h in p)
+    n, t = smp.grow(0.2)
+    assert 1 <= n <= 12 and t > 0
+    cb = bench.cpu_baseline(w, inp, budget_s=0.2)
+    assert cb["cores"] == smp.cores and cb["kind"] == "oracle" and cb["value"] > 0
