@@ -53,6 +53,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "attn_common.cuh"
 #include "attn_tc.h"
 #include "host_cache.h"
 #include "ptx.cuh"
@@ -68,10 +69,6 @@ template <bool kExch, int kBrPerCta>
 constexpr int threads_of() { return 64 + 128 * kBrPerCta + (kExch ? 128 : 0); }  // + MLA exchange warps
 constexpr int kTileSlotBytes = 64 * 128;  // 64 tokens x 64 bf16
 constexpr int kMaxStages = 6;
-constexpr float kRescaleLog2 = 8.f;
-constexpr int kIdAhead = 8;               // page ids read this many pages before their tile
-constexpr int kIdRing = 16;
-static_assert(kIdRing >= kIdAhead + 2, "id ring holds the ids in flight");
 // CTAs per worker.  2: a pair on two SMs, each CTA owning 256 latent dims
 // (four 64-dim blocks).  4 (MLRA-4): one branch of 128 latent dims per CTA,
 // two CTAs resident per SM, each with half of the SM's TMEM and shared memory.
@@ -171,31 +168,6 @@ enum { kEvTma = 0, kEvStageSeen, kEvQkIssued, kEvSReady, kEvSent, kEvRecv, kEvPR
 // wait-site codes recorded with a timeout
 enum { kSiteQEmpty = 1, kSiteStageEmpty, kSiteQFull, kSiteMma, kSiteOFree, kSiteSFull, kSiteXEmpty, kSiteXFull,
        kSitePvDone };
-
-// Cursor over a worker's pages in walk order that reads each page's id from
-// the page table (the producer runs one of these ahead of its loads).
-struct IdFetch {
-  SegWalk w;
-  int p;
-  bool live;
-  __device__ __forceinline__ IdFetch(const WorkerPlan& plan, int B, int maxL, const int* seq_lens)
-      : w(plan, B, maxL), p(0), live(false) {
-    live = w.next(seq_lens);
-    if (live) p = w.pg0;
-  }
-  __device__ __forceinline__ void step(const int* seq_lens) {
-    if (++p >= w.pg1) {
-      live = w.next(seq_lens);
-      if (live) p = w.pg0;
-    }
-  }
-  // id of the current page (not yet waited for), then advance
-  __device__ __forceinline__ int fetch(const int* seq_lens, const int* page_table, int maxp) {
-    const int id = __ldg(page_table + (size_t)w.b * maxp + p);
-    step(seq_lens);
-    return id;
-  }
-};
 
 // One page of online softmax for one row (head) in the log2 domain (the
 // queries arrive pre-multiplied by softmax_scale*log2(e), so the scores are
@@ -922,6 +894,8 @@ bool tc_supported(int dtype, int H, int d_c, int d_r, int n_branch, int /*d_h*/,
 cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop, const int* page_table,
                              const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                              cudaStream_t st, bool pdl) {
+  if (tc_small_supported(a.H, a.n_branch))  // MLA with at most 32 heads: attn_small.cu
+    return launch_attend_tc_small(q_ws, lat, rop, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
   CUtensorMap tq, tqr, tl, tr;
   const bool exch = a.n_branch == 1;
   if (!tmap_2d(&tq, q_ws, (uint64_t)(a.d_c + a.d_r), (uint64_t)a.B * a.H, 64, (uint32_t)a.H) ||
@@ -939,7 +913,7 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
   launch_variant<E, BR, HQ, CTAS>(tq, tqr, tl, tr, page_table, seq_lens, o_part, ml_part, err, a, st, pdl)
   const bool small = a.H <= 32;  // compact query buffers, deeper ring
   switch (a.n_branch) {
-    case 1: return small ? MLRA_LAUNCH(true, 1, 32, 2) : MLRA_LAUNCH(true, 1, 128, 2);
+    case 1: return MLRA_LAUNCH(true, 1, 128, 2);
     case 2: return small ? MLRA_LAUNCH(false, 1, 32, 2) : MLRA_LAUNCH(false, 1, 128, 2);
     // MLRA-4 at full head count: four one-branch CTAs per worker, two per SM
     case 4: return small ? MLRA_LAUNCH(false, 2, 32, 2) : MLRA_LAUNCH(false, 1, 128, 4);
@@ -951,7 +925,8 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
 const char* tc_variant_name(int H, int n_branch) {
   const bool small = H <= 32;
   switch (n_branch) {
-    case 1: return small ? "attend_tc_kernel<mla, cta pair, 32 query rows>" : "attend_tc_kernel<mla, cta pair>";
+    case 1: return small ? "attend_tc_small_kernel<mla, cta pair, head-replicated query>"
+                         : "attend_tc_kernel<mla, cta pair>";
     case 2: return small ? "attend_tc_kernel<mlra-2, cta pair, 32 query rows>" : "attend_tc_kernel<mlra-2, cta pair>";
     case 4: return small ? "attend_tc_kernel<mlra-4, cta pair, 32 query rows>"
                          : "attend_tc_kernel<mlra-4, four ctas, two per sm>";

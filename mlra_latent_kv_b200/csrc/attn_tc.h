@@ -21,6 +21,14 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
                              const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                              cudaStream_t st, bool pdl);
 
+// The MLA kernel for at most 32 heads (attn_small.cu): query rows replicated
+// into every TMEM lane quarter, token-sliced softmax, exact fp32 score
+// exchange, PV with the operands swapped.  launch_attend_tc dispatches to it.
+bool tc_small_supported(int H, int n_branch);
+cudaError_t launch_attend_tc_small(const void* q_ws, const void* lat, const void* rop, const int* page_table,
+                                   const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
+                                   cudaStream_t st, bool pdl);
+
 // Name of the attention kernel variant launch_attend_tc picks for this shape.
 const char* tc_variant_name(int H, int n_branch);
 

@@ -309,3 +309,19 @@ def test_bounded_wait_times_out_and_context_survives():
     w = synth.workload("dsv2_contiguous").with_(B=2, seq_len=130)
     err, tol, *_ = run_case(w, "auto")
     assert err <= tol
+
+
+@pytest.mark.parametrize("name", [w.name for w in synth.WORKLOADS])
+def test_workload_kernel_family(name):
+    """With the default split on the device, kernel AUTO puts every bf16
+    workload on the tcgen05 kernels end to end (a fallback to the CUDA-core
+    kernels would show here); the fp32 tiny workload runs on the CUDA-core
+    kernels, the ones that take fp32."""
+    w = synth.workload(name).with_(B=min(synth.workload(name).B, 8), seq_len=256, seq_len_range=None)
+    s = DecodeSession(w, synth.make_inputs(w))
+    plan = s.plan()
+    assert plan["family"] == ("tcgen05" if w.dtype == "bf16" else "cuda-core"), plan
+    assert plan["splits"] == torch.cuda.get_device_properties(0).multi_processor_count // (2 if w.dtype == "bf16" else 1)
+    s.step()
+    torch.cuda.synchronize()
+    s.check()
