@@ -69,6 +69,11 @@ template <bool kExch, int kBrPerCta>
 constexpr int threads_of() { return 64 + 128 * kBrPerCta + (kExch ? 128 : 0); }  // + MLA exchange warps
 constexpr int kTileSlotBytes = 64 * 128;  // 64 tokens x 64 bf16
 constexpr int kMaxStages = 6;
+// The MLRA-4 four-CTA layout holds only two stages per CTA; its producer also
+// starts page g + kQuadPrefetch towards L2 when it loads page g, so that the
+// load issued when a stage frees mostly hits L2.
+constexpr uint32_t kQuadPrefetch = 2;
+static_assert(kQuadPrefetch < (uint32_t)kIdAhead, "prefetched page ids are already in the id ring");
 // CTAs per worker.  2: a pair on two SMs, each CTA owning 256 latent dims
 // (four 64-dim blocks).  4 (MLRA-4): one branch of 128 latent dims per CTA,
 // two CTAs resident per SM, each with half of the SM's TMEM and shared memory.
@@ -363,6 +368,7 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
       int seg = 0;
       uint32_t g = 0;
       bool ok = true;
+      const uint32_t n_pages = (uint32_t)(plan.end - plan.start);  // pages of this worker
       while (ok && walk.next(seq_lens)) {
         if (seg > 0 && !mbar_wait(smem_u32(&bars->q_empty), (seg - 1) & 1, abort_flag, err, kSiteQEmpty)) break;
         const uint32_t qb = smem_u32(&bars->q_full);
@@ -404,6 +410,13 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
             tma_load_2d(smem_u32(sRope + (g & 1) * L::kRopeTileBytes), &tm_rope, rb, 32 * (int)rank, pg * kPage);
           } else {
             tma_load_2d(smem_u32(tile + kLat * kTileSlotBytes), &tm_rope, fb, 0, pg * kPage);
+          }
+          if (kCtas == 4 && g + kQuadPrefetch < n_pages) {
+            const int pf = id_ring[(g + kQuadPrefetch) % kIdRing];  // written kIdAhead - 1 pages ago
+            if (pf >= 0 && pf < a.num_pages) {
+              for (int s = 0; s < kLat; ++s) tma_prefetch_l2_2d(&tm_lat, 64 * (kLat * (int)rank + s), pf * kPage);
+              tma_prefetch_l2_2d(&tm_rope, 0, pf * kPage);
+            }
           }
           MLRA_TRACE_EV(g, kEvTma);
         }
@@ -887,8 +900,9 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tqr, const 
 }  // namespace
 
 bool tc_supported(int dtype, int H, int d_c, int d_r, int n_branch, int /*d_h*/, int /*d_v*/) {
-  return dtype == 1 && d_c == 512 && d_r == 64 && H >= 1 && H <= kTcHeads &&
-         (n_branch == 1 || n_branch == 2 || n_branch == 4);
+  if (dtype != 1) return false;
+  if (tc_branch_supported(H, d_c, d_r, n_branch)) return true;
+  return d_c == 512 && d_r == 64 && H >= 1 && H <= kTcHeads && (n_branch == 1 || n_branch == 2 || n_branch == 4);
 }
 
 cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop, const int* page_table,
@@ -896,6 +910,8 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
                              cudaStream_t st, bool pdl) {
   if (tc_small_supported(a.H, a.n_branch))  // MLA with at most 32 heads: attn_small.cu
     return launch_attend_tc_small(q_ws, lat, rop, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
+  if (tc_branch_supported(a.H, a.d_c, a.d_r, a.n_branch))  // 128-dim branches: attn_branch.cu
+    return launch_attend_tc_branch(q_ws, lat, rop, page_table, seq_lens, o_part, ml_part, err, a, st, pdl);
   CUtensorMap tq, tqr, tl, tr;
   const bool exch = a.n_branch == 1;
   if (!tmap_2d(&tq, q_ws, (uint64_t)(a.d_c + a.d_r), (uint64_t)a.B * a.H, 64, (uint32_t)a.H) ||
@@ -922,7 +938,8 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
 #undef MLRA_LAUNCH
 }
 
-const char* tc_variant_name(int H, int n_branch) {
+const char* tc_variant_name(int H, int d_c, int n_branch) {
+  if (tc_branch_supported(H, d_c, 64, n_branch)) return "attend_tc_branch_kernel<mla over a 128-dim latent>";
   const bool small = H <= 32;
   switch (n_branch) {
     case 1: return small ? "attend_tc_small_kernel<mla, cta pair, head-replicated query>"

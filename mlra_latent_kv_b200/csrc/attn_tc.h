@@ -29,8 +29,17 @@ cudaError_t launch_attend_tc_small(const void* q_ws, const void* lat, const void
                                    const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                                    cudaStream_t st, bool pdl);
 
+// One 128-dim branch per CTA (attn_branch.cu): the one-branch decode of a
+// 128-dim latent (a branch-parallel MLRA rank's share), 33 to 128 heads.  The
+// grid is n_branch x G CTAs (G page-range workers per branch).
+bool tc_branch_supported(int H, int d_c, int d_r, int n_branch);
+int tc_branch_workers(int sms, int n_branch);
+cudaError_t launch_attend_tc_branch(const void* q_ws, const void* lat, const void* rop, const int* page_table,
+                                    const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
+                                    cudaStream_t st, bool pdl);
+
 // Name of the attention kernel variant launch_attend_tc picks for this shape.
-const char* tc_variant_name(int H, int n_branch);
+const char* tc_variant_name(int H, int d_c, int n_branch);
 
 // Frees the host-side tensor-map cache.
 void tc_shutdown();

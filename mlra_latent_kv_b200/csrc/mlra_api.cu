@@ -112,7 +112,10 @@ mlra_status make_plan(const mlra_dims* d, DecodePlan* p) {
   if (G == 0) {
     const int sms = device_sms();
     if (sms <= 0) return fail(MLRA_ERR_CUDA, "num_splits=0 needs a CUDA device to size the split");
-    G = p->tc ? sms / 2 : sms;
+    // tcgen05: a CTA pair per page range, or (128-dim branches) one CTA per branch and page range
+    G = !p->tc ? sms
+               : (tc_branch_supported(d->H, d->d_c, d->d_r, d->n_branch) ? tc_branch_workers(sms, d->n_branch)
+                                                                          : sms / 2);
   }
   p->G = G;
   p->Hq = d->H;
@@ -233,7 +236,7 @@ mlra_status mlra_describe_plan(const mlra_dims* dims, char* buf, size_t buf_len)
   const int n = snprintf(buf, buf_len,
                          "family=%s;splits=%d;kernels=%d;absorb=%s;attention=%s;combine=%s;upproj=%s", family, p.G,
                          2 + (tc_upproj ? 1 : 2), tc_absorb ? "absorb_tc_kernel" : "absorb_kernel",
-                         p.tc ? tc_variant_name(d->H, d->n_branch) : "attend_simt_kernel",
+                         p.tc ? tc_variant_name(d->H, d->d_c, d->n_branch) : "attend_simt_kernel",
                          tc_upproj ? "fused into combine_upproj_tc_kernel" : "combine_kernel",
                          tc_upproj ? "combine_upproj_tc_kernel" : "upproj_kernel");
   if (n < 0 || (size_t)n >= buf_len) return fail(MLRA_ERR_INVALID_ARG, "buf too small (%d bytes needed)", n + 1);

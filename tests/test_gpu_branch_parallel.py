@@ -23,6 +23,8 @@ def test_branch_parallel_shares_sum_to_the_mlra4_decode(H):
     total = None
     for r in range(w.n_branch):
         bp = BranchParallelDecode(w, inp, r)
+        plan = bp.sess.plan()
+        assert plan["family"] == "tcgen05" and "128-dim latent" in plan["attention"], plan
         part = bp.partial().float()
         torch.cuda.synchronize()
         bp.sess.check()

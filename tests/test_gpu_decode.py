@@ -321,7 +321,10 @@ def test_workload_kernel_family(name):
     s = DecodeSession(w, synth.make_inputs(w))
     plan = s.plan()
     assert plan["family"] == ("tcgen05" if w.dtype == "bf16" else "cuda-core"), plan
-    assert plan["splits"] == torch.cuda.get_device_properties(0).multi_processor_count // (2 if w.dtype == "bf16" else 1)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # page ranges: a CTA pair each (tcgen05), one CTA per branch and range (128-dim branches), one CTA (CUDA cores)
+    per = 1 if w.dtype != "bf16" else (w.n_branch if "branch" in plan["attention"] else 2)
+    assert plan["splits"] == sms // per, plan
     s.step()
     torch.cuda.synchronize()
     s.check()
