@@ -120,7 +120,8 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": sorted(self.reasons)}
 
 
-ATTN_SOURCES = ("attn_tc.cu", "attn_tc.h", "ptx.cuh", "common.cuh", "launch.h", "host_cache.cu", "host_cache.h")
+ATTN_SOURCES = ("attn_tc.cu", "attn_small.cu", "attn_branch.cu", "attn_common.cuh", "attn_tc.h", "ptx.cuh",
+                "common.cuh", "launch.h", "host_cache.cu", "host_cache.h")
 
 
 def source_digest() -> str:
