@@ -21,10 +21,11 @@
 //     send each page's partial to the peer through distributed shared memory
 //     as soon as QK^T has produced it, as the row's maximum r over the page's
 //     tokens (fp32) and each score's offset from it, s - r, rounded to fp16.
-//     Both CTAs then form (r_0 + r_1) + (f16(s_0 - r_0) + f16(s_1 - r_1)):
-//     fp32 addition commutes, so they hold the same bits and compute identical
-//     softmax weights, and the rounding error of a score is 2^-11 of its
-//     distance below its row's page maximum, however large the logits.
+//     Both CTAs then form (r_0 + r_1) + (f16(s_0 - r_0) + f16(s_1 - r_1)),
+//     the offsets added as an fp16 pair: addition commutes, so they hold the
+//     same bits and compute identical softmax weights, and the rounding error
+//     of a score is a few 2^-11 of its distance below its row's page maximum,
+//     however large the logits.
 //   * MLRA with 2 or 4 branches: the branches of a CTA are wholly its own, so
 //     the CTAs of a worker never talk; each adds the full rope score to its
 //     branches.  MLRA-4 with more than 32 heads runs four CTAs per worker, one
@@ -219,21 +220,35 @@ __device__ __forceinline__ bool softmax_page(float (&s)[64], int valid, bool fir
 // Maximum of a row's scores over the page's first `valid` tokens (the exact
 // value does not depend on the order, so the exchange warp, which holds the
 // scores as two 32-column halves, and the softmax warp agree on it).
+// (Full pages, all but a sequence's last, take the unmasked branch.)
 __device__ __forceinline__ float row_max_valid(const uint32_t (&lo)[32], const uint32_t (&hi)[32], int valid) {
   float m8[8];
+  if (valid >= 64) {
 #pragma unroll
-  for (int n = 0; n < 64; ++n) {
-    const float v = n < valid ? __uint_as_float(n < 32 ? lo[n] : hi[n - 32]) : -INFINITY;
-    m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+    for (int n = 0; n < 64; ++n) {
+      const float v = __uint_as_float(n < 32 ? lo[n] : hi[n - 32]);
+      m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+    }
+  } else {
+#pragma unroll
+    for (int n = 0; n < 64; ++n) {
+      const float v = n < valid ? __uint_as_float(n < 32 ? lo[n] : hi[n - 32]) : -INFINITY;
+      m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+    }
   }
   return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
 __device__ __forceinline__ float row_max_valid(const float (&s)[64], int valid) {
   float m8[8];
+  if (valid >= 64) {
 #pragma unroll
-  for (int n = 0; n < 64; ++n) {
-    const float v = n < valid ? s[n] : -INFINITY;
-    m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+    for (int n = 0; n < 64; ++n) m8[n & 7] = n < 8 ? s[n] : fmaxf(m8[n & 7], s[n]);
+  } else {
+#pragma unroll
+    for (int n = 0; n < 64; ++n) {
+      const float v = n < valid ? s[n] : -INFINITY;
+      m8[n & 7] = n < 8 ? v : fmaxf(m8[n & 7], v);
+    }
   }
   return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
@@ -747,8 +762,9 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
           }
           if (row == 0) MLRA_TRACE_EV(g, kEvRecv);
           if (real) {
-            // s = (r_own + r_peer) + (f16(s_own - r_own) + f16(s_peer - r_peer)); each sum has the
-            // same operands on both CTAs, in the other order, so both get the same bits
+            // s = (r_own + r_peer) + (f16(s_own - r_own) + f16(s_peer - r_peer)), the offsets added as an
+            // fp16 pair; each sum has the same operands on both CTAs, in the other order, so both get the
+            // same bits (the exchange warp packed f16(s_own - r_own) the same way for the peer)
             const float r_own = row_max_valid(cur, valid);
             const float r_sum = r_own + sXR[row];
 #pragma unroll
@@ -757,11 +773,10 @@ __global__ void __launch_bounds__(threads_of<kExch, kBrPerCta>(), min_blocks<kCt
               const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const float2 mine =
-                    unpack_f16x2(pack_f16x2(cur[8 * q + 2 * j] - r_own, cur[8 * q + 2 * j + 1] - r_own));
-                const float2 theirs = unpack_f16x2(w[j]);
-                cur[8 * q + 2 * j] = r_sum + (mine.x + theirs.x);
-                cur[8 * q + 2 * j + 1] = r_sum + (mine.y + theirs.y);
+                const float2 d = unpack_f16x2(
+                    add_f16x2(pack_f16x2(cur[8 * q + 2 * j] - r_own, cur[8 * q + 2 * j + 1] - r_own), w[j]));
+                cur[8 * q + 2 * j] = r_sum + d.x;
+                cur[8 * q + 2 * j + 1] = r_sum + d.y;
               }
             }
           }

@@ -356,6 +356,13 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
   return f;
 }
 
+// fp16x2 addition, round to nearest even (commutative: a + b and b + a give the same bits)
+__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
