@@ -182,6 +182,39 @@ MLRA_API mlra_status mlra_decode_host(const mlra_dims* dims, const void* h_q_nop
  * the library's own kernels serve the decode step of the method above. */
 MLRA_API mlra_status mlra_describe_plan(const mlra_dims* dims, char* buf, size_t buf_len);
 
+/* Sequence-sharded decode across GPUs (long contexts).  When the cached
+ * tokens of every sequence are spread over R GPUs, each GPU attends its own
+ * token range: mlra_attend_partial runs the decode's absorption and split-KV
+ * attention on that GPU's cache and writes, per (sequence, head, branch), the
+ * latent output normalised over its tokens and the log-sum-exp of its scores
+ * in base 2 (the scores already carry softmax_scale * log2(e)):
+ *   o   [B, H, d_c] fp32     o[b,h,br block] = sum_t p_t c_t,br / sum_t p_t
+ *   lse [B, n_branch, H] fp32   log2 sum_t 2^(s_t)   (-inf and o = 0 when the
+ *                                                     GPU holds no token of b)
+ * After the R partials are gathered (the caller's all-gather, in a fixed rank
+ * order), mlra_merge_upproj weighs part r by 2^(lse_r - lse) with
+ * lse = log2 sum_r 2^(lse_r) -- the softmax over all of the sequence's tokens
+ * -- folds in branch_scale and applies W_UV:
+ *   o_parts [R, B, H, d_c] fp32, lse_parts [R, B, n_branch, H] fp32,
+ *   out [B, H, d_v] (dtype), workspace >= mlra_merge_workspace_bytes(dims).
+ * Positions: a GPU's cache and page table address its own tokens from 0, but
+ * the stored rope keys must be rotated at their absolute positions (write the
+ * cache through a page table indexed by absolute page, then attend through
+ * that table's rows shifted to the GPU's first page); q_pos is absolute.
+ * mlra_attend_partial takes the decode's arguments and workspace
+ * (mlra_workspace_bytes) minus W_UV and out.  Method: yololab.net,
+ * "超越 GQA 的推理革命…", section "矩陣吸收" (W_UV after attention); the merge
+ * is the split-KV combine of the single-GPU path applied across GPUs. */
+MLRA_API mlra_status mlra_attend_partial(const mlra_dims* dims, const void* q_nope, const void* q_rope,
+                                         const int32_t* q_pos, const void* W_UK, const void* latent_cache,
+                                         const void* rope_cache, const int32_t* page_table,
+                                         const int32_t* seq_lens, float* o, float* lse, void* workspace,
+                                         size_t workspace_bytes, cudaStream_t stream);
+MLRA_API size_t mlra_merge_workspace_bytes(const mlra_dims* dims);
+MLRA_API mlra_status mlra_merge_upproj(const mlra_dims* dims, int n_parts, const float* o_parts,
+                                       const float* lse_parts, const void* W_UV, void* out, void* workspace,
+                                       size_t workspace_bytes, cudaStream_t stream);
+
 /* Bytes of workspace latent_append needs for hidden width d_model. */
 MLRA_API size_t latent_append_workspace_bytes(const mlra_dims* dims, int d_model);
 

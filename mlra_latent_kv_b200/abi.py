@@ -61,6 +61,9 @@ SIGNATURES = {
     "latent_store": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _I32P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "latent_append_noalloc": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _I32P, _I32P, _P, _P, _P]),
     "mlra_describe_plan": (ctypes.c_int, [_DIMS, ctypes.c_char_p, _SZ]),
+    "mlra_attend_partial": (ctypes.c_int, [_DIMS, _P, _P, _I32P, _P, _P, _P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
+    "mlra_merge_workspace_bytes": (_SZ, [_DIMS]),
+    "mlra_merge_upproj": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _P, _P, _SZ, _P]),
     "mlra_check_status": (ctypes.c_int, [_P, _P]),
     "mlra_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_longlong, _P]),
     "mlra_last_error": (ctypes.c_char_p, []),
@@ -118,6 +121,29 @@ def describe_plan(dims: Dims) -> dict:
     out = dict(kv.split("=", 1) for kv in buf.value.decode().split(";"))
     out["splits"], out["kernels"] = int(out["splits"]), int(out["kernels"])
     return out
+
+
+def attend_partial(dims, q_nope, q_rope, q_pos, W_UK, latent_cache, rope_cache, page_table, seq_lens, o, lse,
+                   workspace, stream=None):
+    """A sequence-sharded rank's partial: o [B,H,d_c] fp32 and lse [B,n_branch,H] fp32 (see include/mlra.h)."""
+    _check(lib().mlra_attend_partial(ctypes.byref(dims), _ptr(q_nope), _ptr(q_rope), _ptr(q_pos), _ptr(W_UK),
+                                     _ptr(latent_cache), _ptr(rope_cache), _ptr(page_table), _ptr(seq_lens),
+                                     _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)))
+
+
+def merge_workspace_bytes(dims: Dims) -> int:
+    n = lib().mlra_merge_workspace_bytes(ctypes.byref(dims))
+    if n == 0:
+        raise MlraError(1, last_error())
+    return int(n)
+
+
+def merge_upproj(dims, o_parts, lse_parts, W_UV, out, workspace, stream=None):
+    """Merges R gathered partials ([R,B,H,d_c], [R,B,n_branch,H]) and applies W_UV into out."""
+    _check(lib().mlra_merge_upproj(ctypes.byref(dims), int(o_parts.shape[0]), _ptr(o_parts), _ptr(lse_parts),
+                                   _ptr(W_UV), _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def workspace_bytes(dims: Dims) -> int:

@@ -46,6 +46,12 @@ cudaError_t launch_combine(bool out_bf16, const float* o_part, const float* ml_p
 cudaError_t launch_upproj(int dtype, bool in_bf16, const void* o_lat, const void* W_UV, void* out, const UpArgs& a,
                           cudaStream_t st);
 
+// sequence-sharded decode (seq_parallel.cu): a rank's partial, and the merge of R gathered partials
+cudaError_t launch_partial(const float* o_part, const float* ml_part, const int* seq_lens, float* o_out,
+                           float* lse_out, const CombineArgs& a, cudaStream_t st);
+cudaError_t launch_merge(bool out_bf16, const float* o_parts, const float* lse_parts, void* o_lat, int R, int B, int H,
+                         int d_c, int n_branch, float branch_scale, cudaStream_t st);
+
 cudaError_t launch_append(int dtype, const void* h, const void* W_DKV, const void* W_KR, const int* pos,
                           const int* page_table, void* lat, void* rop, float* part, int* err, const AppendArgs& a,
                           const RopeTable& tab, cudaStream_t st);

@@ -134,16 +134,26 @@ mlra_status make_plan(const mlra_dims* d, DecodePlan* p) {
   return MLRA_OK;
 }
 
+// The rank's partial of a sequence-sharded decode, written instead of `out`
+// when decode_impl is called with one: o [B,H,d_c] fp32, lse [B,n_branch,H].
+struct PartialOut {
+  float* o;
+  float* lse;
+};
+
 mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, const void* q_rope,
                         const int32_t* q_pos, const void* W_UK, const void* W_UV, const void* latent_cache,
                         const void* rope_cache, const int32_t* page_table, const int32_t* seq_lens, void* out,
-                        void* workspace, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* ev) {
+                        void* workspace, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* ev,
+                        const PartialOut* part = nullptr) {
   DecodePlan p;
   mlra_status st = make_plan(d, &p);
   if (st != MLRA_OK) return st;
   if (mla_only && d->n_branch != 1) return fail(MLRA_ERR_INVALID_ARG, "mla_decode needs n_branch=1 (use mlra_decode)");
-  const void* ptrs[] = {q_nope, q_rope, W_UK, W_UV, latent_cache, rope_cache, out, workspace};
-  const char* names[] = {"q_nope", "q_rope", "W_UK", "W_UV", "latent_cache", "rope_cache", "out", "workspace"};
+  const void* ptrs[] = {q_nope, q_rope, W_UK, part ? part->o : W_UV, latent_cache, rope_cache,
+                        part ? part->lse : out, workspace};
+  const char* names[] = {"q_nope", "q_rope", "W_UK", part ? "o" : "W_UV", "latent_cache", "rope_cache",
+                         part ? "lse" : "out", "workspace"};
   for (int i = 0; i < 8; ++i) {
     if (!ptrs[i]) return fail(MLRA_ERR_INVALID_ARG, "%s is NULL", names[i]);
     if (!aligned(ptrs[i], 16)) return fail(MLRA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
@@ -200,6 +210,13 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   }
   if (ev) record_event(ev[2], stream);
+
+  if (part) {  // a sequence-sharded rank: its partial instead of the combine and up-projection
+    CombineArgs ca{d->B, d->H, d->d_c, d->n_branch, p.G, d->max_pages_per_seq, 1.0f};
+    e = launch_partial(o_part, ml_part, seq_lens, part->o, part->lse, ca, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "partial launch");
+    return MLRA_OK;
+  }
 
   if (tc_upproj) {  // combine fused into the up-projection: stage 3 is empty
     if (ev) record_event(ev[3], stream);
@@ -340,6 +357,45 @@ mlra_status mlra_decode_host(const mlra_dims* dims, const void* h_q_nope, const 
   cudaError_t e3 = cudaMemcpyAsync(h_out, ws + h.out, (size_t)d->B * d->H * d->d_v * e, cudaMemcpyDeviceToHost,
                                    stream);
   if (e3 != cudaSuccess) return cuda_fail(e3, "device-to-host copy");
+  return MLRA_OK;
+}
+
+mlra_status mlra_attend_partial(const mlra_dims* dims, const void* q_nope, const void* q_rope, const int32_t* q_pos,
+                                const void* W_UK, const void* latent_cache, const void* rope_cache,
+                                const int32_t* page_table, const int32_t* seq_lens, float* o, float* lse,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const PartialOut part{o, lse};
+  return decode_impl(dims, false, q_nope, q_rope, q_pos, W_UK, nullptr, latent_cache, rope_cache, page_table,
+                     seq_lens, nullptr, workspace, workspace_bytes, stream, nullptr, &part);
+}
+
+size_t mlra_merge_workspace_bytes(const mlra_dims* dims) {
+  if (check_dims(dims) != MLRA_OK) return 0;
+  return round_up((size_t)dims->B * dims->H * dims->d_c * (dims->dtype == MLRA_BF16 ? 2 : 4), 256);
+}
+
+mlra_status mlra_merge_upproj(const mlra_dims* dims, int n_parts, const float* o_parts, const float* lse_parts,
+                              const void* W_UV, void* out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  mlra_status st = check_dims(dims);
+  if (st != MLRA_OK) return st;
+  const mlra_dims* d = dims;
+  if (n_parts < 1) return fail(MLRA_ERR_INVALID_ARG, "n_parts must be >= 1");
+  const void* ptrs[] = {o_parts, lse_parts, W_UV, out, workspace};
+  const char* names[] = {"o_parts", "lse_parts", "W_UV", "out", "workspace"};
+  for (int i = 0; i < 5; ++i) {
+    if (!ptrs[i]) return fail(MLRA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned(ptrs[i], 16)) return fail(MLRA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  const size_t need = mlra_merge_workspace_bytes(d);
+  if (workspace_bytes < need) return fail(MLRA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  const bool bf16 = d->dtype == MLRA_BF16;
+  cudaError_t e = launch_merge(bf16, o_parts, lse_parts, workspace, n_parts, d->B, d->H, d->d_c, d->n_branch,
+                               d->branch_scale, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  UpArgs ua{d->B, d->H, d->d_c, d->d_v};
+  e = launch_upproj(d->dtype, bf16, workspace, W_UV, out, ua, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "up-projection launch");
   return MLRA_OK;
 }
 

@@ -27,6 +27,7 @@ static void* const entry_points[] = {
     (void*)latent_append,         (void*)latent_store,         (void*)latent_append_noalloc,
     (void*)mlra_selftest_wait_timeout, (void*)mlra_check_status, (void*)mlra_last_error,
     (void*)mlra_shutdown,         (void*)mlra_version,          (void*)mlra_describe_plan,
+    (void*)mlra_attend_partial,   (void*)mlra_merge_workspace_bytes, (void*)mlra_merge_upproj,
 };
 
 static mlra_dims dims_dsv2(void) {
