@@ -10,9 +10,10 @@
 // for B rows), so they run "swap-AB": the weight is the M x K operand (M =
 // latent or value dims, MN-major straight from its row-major layout by TMA),
 // the batch is N (padded to a multiple of 16 with TMA zero fill), and one CTA
-// per (head, 128-row M tile) streams its weight slice once.  The combine is
-// fused into the up-projection: the CTA of head h merges the partials of every
-// sequence into bf16 rows of the MMA's B operand in shared memory, so o_lat
+// per (head, 128-row M tile) streams its weight slice once (the up-projection:
+// once per block of 16 sequences, the repeats from L2).  The combine is fused
+// into the up-projection: the CTA of head h merges the partials of its
+// sequences into bf16 rows of the MMA's B operand in shared memory, so o_lat
 // never goes to HBM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -180,13 +181,17 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------------------------------
 // a4 + a5: split combine fused into the output up-projection.
-// grid (H, d_v / 128), block 512.
-//   A (M = 128 value dims, K = d_c) = W_UV[h][:, m0:m0+128]   MN-major (TMA)
-//   B (N = Bp batch rows, K = d_c)  = o_lat[:, h, :] built here in smem:
+// grid (H, d_v / 128, ceil(B / kCuRows)), block 512: a CTA takes one head, 128
+// value dims and a block of kCuRows sequences, so that a few heads still fill
+// the GPU (at H = 32 one CTA per head would leave most SMs idle, each of its
+// CTAs streaming a whole head's partials).
+//   A (M = 128 value dims, K = d_c)      = W_UV[h][:, m0:m0+128]  MN-major (TMA)
+//   B (N = kCuRows batch rows, K = d_c)  = o_lat[b0 + n, h, :] built here in smem:
 //       o_lat[b, h, br cols] = branch_scale * sum_s 2^(m_s - M) o_s / L
-//   D (TMEM, 128 lanes x Bp)        -> out[b][h][m0 + lane] (bf16)
+//   D (TMEM, 128 lanes x kCuRows)        -> out[b][h][m0 + lane] (bf16)
 // ---------------------------------------------------------------------------
 constexpr int kCuThreads = 512;
+constexpr int kCuRows = 16;      // sequences per CTA (the MMA's N)
 constexpr int kPieceUnroll = 4;  // partials of a row fetched together
 
 __global__ void __launch_bounds__(kCuThreads, 1)
@@ -197,9 +202,9 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int a_bytes = 2 * a.K * 128;             // K = d_c rows, two 64-column M blocks
   const int n_ml = (a.G + a.B - 1) * a.n_branch;  // (slot, branch) pairs
-  uint8_t* sB = smem + a_bytes;                  // d_c/64 blocks of Bp rows
+  uint8_t* sB = smem + a_bytes;                  // d_c/64 blocks of kCuRows rows
   uint8_t* sA = smem;
-  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * a.Bp * 128);  // [slot][n_branch] piece weights
+  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * kCuRows * 128);  // [slot][n_branch] piece weights
   float* s_m = s_wt + n_ml;                                              // [slot][n_branch] running max
   float* s_l = s_m + n_ml;                                               // [slot][n_branch] sum
   int* s_c0 = reinterpret_cast<int*>(s_l + n_ml);
@@ -209,9 +214,10 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   __shared__ long long s_T;
-  const int h = blockIdx.x, m0 = blockIdx.y * 128;
+  const int h = blockIdx.x, m0 = blockIdx.y * 128, b0 = blockIdx.z * kCuRows;
+  const int nb = min(kCuRows, a.B - b0);  // sequences of this CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = tmem_cols_for(a.Bp);
+  const uint32_t ncols = tmem_cols_for(kCuRows);
   const int maxL = a.maxp * kPage;
   GEMM_TRACE(1, 0);
   if (threadIdx.x == 0) {
@@ -265,8 +271,13 @@ __global__ void __launch_bounds__(kCuThreads, 1)
       s_ne[c] = worker_start(c, T, a.G) != worker_start(c + 1, T, a.G) ? 1 : 0;
   }
   grid_dep_wait();  // the partials come from the attention kernel
-  // (m, l) of every slot of this head, all loads in flight at once
-  for (int i = threadIdx.x; i < n_ml; i += blockDim.x) {
+  // (m, l) of the slots of this CTA's sequences, all loads in flight at once
+  // (slot c + b for worker c; the sequences b0 .. b0 + nb - 1 use slots
+  // s_c0[b0] + b0 .. s_c1[b0 + nb - 1] + b0 + nb - 1)
+  const int slot_lo = nb > 0 ? s_c0[b0] + b0 : 0;
+  int slot_hi = slot_lo - 1;
+  for (int b = b0; b < b0 + nb; ++b) slot_hi = max(slot_hi, s_c1[b] + b);
+  for (int i = slot_lo * a.n_branch + threadIdx.x; i < (slot_hi + 1) * a.n_branch; i += blockDim.x) {
     const size_t base = (size_t)i * 2;
     s_m[i] = ml_part[(base + 0) * a.H + h];
     s_l[i] = ml_part[(base + 1) * a.H + h];
@@ -274,8 +285,8 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   __syncthreads();
   GEMM_TRACE(1, 1);
   // per (b, branch): weight of each piece, 2^(m_s - M) * branch_scale / L
-  for (int idx = threadIdx.x; idx < a.B * a.n_branch; idx += blockDim.x) {
-    const int b = idx / a.n_branch, br = idx % a.n_branch;
+  for (int idx = threadIdx.x; idx < nb * a.n_branch; idx += blockDim.x) {
+    const int b = b0 + idx / a.n_branch, br = idx % a.n_branch;
     const int c0 = s_c0[b], c1 = s_c1[b];
     float M = -INFINITY;
     for (int c = c0; c <= c1; ++c)
@@ -299,16 +310,17 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   // the partials of up to kPieceUnroll pieces of both before using any.
   const int chunks = a.K / 8;
   const int d_cb = a.K / a.n_branch;
-  const int n_items = a.Bp * chunks;
+  const int n_items = kCuRows * chunks;
   for (int base = threadIdx.x; base < n_items; base += 2 * blockDim.x) {
-    int bq[2], chq[2], c0q[2], c1q[2], brq[2];
+    int rq[2], bq[2], chq[2], c0q[2], c1q[2], brq[2];  // local row, sequence, chunk, workers, branch
     float acc[2][8];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int idx = base + u * blockDim.x;
-      bq[u] = idx < n_items ? idx / chunks : a.Bp;
+      rq[u] = idx < n_items ? idx / chunks : kCuRows;
+      bq[u] = b0 + rq[u];
       chq[u] = idx % chunks;
-      const bool row = bq[u] < a.B;
+      const bool row = rq[u] < nb;
       c0q[u] = row ? s_c0[bq[u]] : 0;
       c1q[u] = row ? s_c1[bq[u]] : -1;
       brq[u] = (chq[u] * 8) / d_cb;
@@ -351,13 +363,13 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      if (bq[u] >= a.Bp) continue;
-      uint4 pk;
+      if (rq[u] >= kCuRows) continue;
+      uint4 pk;  // rows past the batch are zero (no pieces, weights 0)
       pk.x = pack_bf16x2(acc[u][0], acc[u][1]);
       pk.y = pack_bf16x2(acc[u][2], acc[u][3]);
       pk.z = pack_bf16x2(acc[u][4], acc[u][5]);
       pk.w = pack_bf16x2(acc[u][6], acc[u][7]);
-      *reinterpret_cast<uint4*>(sB + (chq[u] / 8) * a.Bp * 128 + sw128_off(bq[u], chq[u] % 8)) = pk;
+      *reinterpret_cast<uint4*>(sB + (chq[u] / 8) * kCuRows * 128 + sw128_off(rq[u], chq[u] % 8)) = pk;
     }
   }
   fence_proxy_async_smem();
@@ -367,10 +379,10 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     if (mbar_wait(smem_u32(&full_bar), 0, &abort_flag, err, 22)) {
       GEMM_TRACE(1, 4);
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, a.Bp, true, false);
+      const uint32_t idesc = idesc_bf16_f32(128, kCuRows, true, false);
       const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
       const uint64_t bd0 = sdesc_sw128(smem_u32(sB), 16, 1024);
-      const uint64_t bkb = (uint64_t)((a.Bp * 128) >> 4);
+      const uint64_t bkb = (uint64_t)((kCuRows * 128) >> 4);
       for (int kb = 0; kb < a.K / 64; ++kb) {
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
@@ -384,16 +396,13 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     GEMM_TRACE(1, 5);
     tc_fence_after();
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    for (int cc = 0; cc < a.Bp; cc += 32) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + cc, v);
+    static_assert(kCuRows == 16, "one 16-column TMEM load per lane quarter");
+    uint32_t v[16];
+    tmem_ld16(tmem + lane_off, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int b = cc + j;
-        if (b < a.B)
-          out[((size_t)b * a.H + h) * a.N_out + m0 + warp * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j]));
-      }
-    }
+    for (int j = 0; j < kCuRows; ++j)
+      if (j < nb)
+        out[((size_t)(b0 + j) * a.H + h) * a.N_out + m0 + warp * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j]));
   }
   tc_fence_before();
   __syncthreads();
@@ -413,16 +422,16 @@ bool absorb_tc_supported(int dtype, int B, int d_h, int d_c) {
 
 int batch_pad(int B) { return B <= 16 ? 16 : (B + 15) / 16 * 16; }
 
-// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B), d_c/64 x Bp x 128 B
-// of o_lat rows, the (m, l, weight) of every slot and branch, two ints per row,
-// one flag per worker
+// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B), d_c/64 x kCuRows x
+// 128 B of o_lat rows, the (m, l, weight) of every slot and branch, two ints
+// per sequence, one flag per worker
 static size_t upproj_smem_bytes(int B, int d_c, int G, int n_branch) {
-  return 1024 + (size_t)2 * d_c * 128 + (size_t)(d_c / 64) * batch_pad(B) * 128 +
+  return 1024 + (size_t)2 * d_c * 128 + (size_t)(d_c / 64) * kCuRows * 128 +
          (size_t)3 * (G + B) * n_branch * 4 + (size_t)2 * B * 4 + (size_t)G * 4;
 }
 
 bool upproj_tc_supported(int dtype, int B, int d_c, int d_v, int G, int n_branch) {
-  return dtype == 1 && B >= 1 && B <= 96 && d_c % 64 == 0 && d_c <= 512 && (d_c <= 256 || d_c % 256 == 0) &&
+  return dtype == 1 && B >= 1 && d_c % 64 == 0 && d_c <= 512 && (d_c <= 256 || d_c % 256 == 0) &&
          d_v % 128 == 0 && upproj_smem_bytes(B, d_c, G, n_branch) <= 232448;
 }
 
@@ -450,7 +459,7 @@ cudaError_t launch_combine_upproj_tc(const float* o_part, const float* ml_part, 
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(combine_upproj_tc_kernel), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.H, a.N_out / 128, 1);
+  cfg.gridDim = dim3(a.H, a.N_out / 128, (a.B + kCuRows - 1) / kCuRows);
   cfg.blockDim = dim3(kCuThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
