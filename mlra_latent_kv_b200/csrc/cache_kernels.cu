@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "ptx.cuh"
 
 namespace mlra {
 
@@ -17,9 +18,12 @@ namespace mlra {
 //   part[ks, b, j] = sum_{k in chunk ks} h[b, k] * Wcat[k, j],   Wcat = [W_DKV | W_KR]
 // grid (KS) chunks of 64 weight rows.  A thread owns kCG adjacent columns (one
 // 16-byte load per weight row) in one of kRG row groups (rows rg, rg + kRG,
-// ...), issues all its row loads before using them, and the row groups are
-// summed in a fixed order through shared memory.  Batch rows are taken kAppendB
-// at a time from shared memory.  Weight rows are read exactly once.
+// ...), issues its row loads 16 at a time (8 for fp32) before using any, so a
+// bf16 chunk costs one memory round trip, and the row groups are summed
+// in a fixed order through shared memory.  Batch rows are taken kAppendB at a
+// time from shared memory.  Weight rows are read exactly once.  The finalize
+// kernel may launch as soon as this grid starts (programmatic dependent
+// launch); it waits for this grid's sums before reading them.
 // ---------------------------------------------------------------------------
 constexpr int kAppendRows = 64;
 constexpr int kAppendB = 4;
@@ -45,6 +49,7 @@ __global__ void __launch_bounds__(append_threads<kCG>()) append_partial_kernel(c
   const int n_cg = W / kCG;
   const int cg = threadIdx.x % n_cg, rg = threadIdx.x / n_cg;
   const int j = cg * kCG;
+  ptx::grid_dep_launch();
   const T* wp;
   int ld;
   if (j < a.d_c) {
@@ -66,7 +71,8 @@ __global__ void __launch_bounds__(append_threads<kCG>()) append_partial_kernel(c
     for (int c = 0; c < kCG; ++c)
 #pragma unroll
       for (int i = 0; i < kAppendB; ++i) acc[c][i] = 0.f;
-    constexpr int kBatch = 8;  // weight rows in flight per thread
+    constexpr int kMaxBatch = sizeof(T) == 2 ? 16 : 8;  // 16-byte loads: up to 16 rows in flight at once
+    constexpr int kBatch = kRowsPerRG < kMaxBatch ? kRowsPerRG : kMaxBatch;
 #pragma unroll 1
     for (int r0 = 0; r0 < kRowsPerRG; r0 += kBatch) {
       Vec wv[kBatch];
@@ -134,6 +140,7 @@ __global__ void append_finalize_kernel(const float* __restrict__ part, const int
   const int pairs = W / 2;
   const int lane = threadIdx.x & 31;
   const int idx = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  ptx::grid_dep_wait();  // the partial sums come from the previous kernel
   if (idx >= a.B * pairs) return;
   const int b = idx / pairs, j = 2 * (idx % pairs);
   float x0 = 0.f, x1 = 0.f;
@@ -192,9 +199,21 @@ static cudaError_t launch_append_t(const void* h, const void* W_DKV, const void*
     if (e != cudaSuccess) return e;
   }
   k1<<<a.KS, thr, smem, st>>>((const T*)h, (const T*)W_DKV, (const T*)W_KR, part, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the finalize kernel as a programmatic dependent of the partial sums
   const int n2 = a.B * (W / 2);
-  append_finalize_kernel<T><<<(n2 + 7) / 8, 256, 0, st>>>(part, pos, page_table, (T*)lat, (T*)rop, err, a, tab);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((n2 + 7) / 8, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, append_finalize_kernel<T>, (const float*)part, pos, page_table, (T*)lat, (T*)rop,
+                            err, a, tab);
 }
 
 cudaError_t launch_append(int dtype, const void* h, const void* W_DKV, const void* W_KR, const int* pos,
