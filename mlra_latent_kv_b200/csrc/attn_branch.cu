@@ -1,7 +1,5 @@
-// tcgen05 split-KV latent attention, one 128-dim branch per CTA (sm_100a):
-// the one-branch (MLA) decode of a 128-dim latent that each rank of a
-// branch-parallel MLRA group runs (see tc_branch_supported for why MLRA-4 over
-// a 512-dim latent is sent to the four-CTA layout instead).
+// tcgen05 split-KV latent attention, one 128-dim branch per CTA (sm_100a),
+// over units of two pages.
 //
 // Method: wispaper.ai, "MLRA：突破 MLA 并行瓶颈…", section "2.1 架构拆解":
 // each branch br attends with its own softmax over its own block of the
@@ -15,21 +13,23 @@
 // Design (B200, up to 128 heads):
 //   * A CTA takes one branch of one page range; one CTA per SM.  The grid is
 //     n_branch x G CTAs: CTA (br, c) attends branch br over worker c's pages.
-//   * The branch's query (128 latent dims and the 64 rope dims of every head)
-//     lives in TMEM beside O (128 columns) and a ring of four S buffers, so
-//     shared memory holds only pages: up to nine stages of 24 KB (the
-//     branch's two 64-dim latent blocks and the 64-dim rope block).
-//   * QK^T (M = 128 heads, N = 64 tokens, A from TMEM) and PV (A = P in TMEM,
-//     B = the page's latent read MN-major, N = 128) are issued by two warps,
-//     so a PV whose P is ready never waits behind the next page's QK^T issue.
-//   * Four softmax warps per TMEM lane quarter split each page's 64 tokens in
-//     16-token slices: 16 scores per thread, and four warps per SM
-//     sub-partition to hide each other's latency.  The four agree on each
-//     page's row maximum through shared memory (an mbarrier per lane quarter
-//     and page), write their slices of P (bf16) over S, and share the rare O
-//     rescale.
-//   * Four query warps load each piece's query into TMEM once the previous
-//     piece's last QK^T has completed.
+//   * Pages go through the CTA in units of two (128 tokens; a piece's last
+//     unit may hold one page).  A unit's pages sit next to each other in
+//     shared memory, so QK^T is one N = 128 MMA per 16 dims for both pages:
+//     a tcgen05 MMA of N <= 64 costs at least ~45 cycles whatever its size,
+//     and N = 128 runs at the full rate.  The unit is also the step of every
+//     barrier hand-off, which halves them against a page-sized step.
+//   * The branch's query (128 latent dims and 64 rope dims per head) lives in
+//     TMEM beside O (128 columns) and two S buffers of 128 columns, so shared
+//     memory holds only the unit ring: four units of 48 KB.
+//   * QK^T (M = 128 heads, N = 128 tokens, A = the query in TMEM) and PV (A =
+//     P in TMEM, B = the unit's latent read MN-major, N = 128 dims) are issued
+//     by two warps.
+//   * Softmax: per TMEM lane quarter, four warps, one per 32 tokens of the
+//     unit; they agree on the unit's row maximum through shared memory, and
+//     each writes the P (bf16) of its tokens over its own score columns.  O is
+//     rescaled only when the running max grows by more than 2^8.  The first
+//     warp of each quarter also loads the query rows into TMEM per piece.
 //   * Rows past the sequence end in the last page are zeroed in shared memory
 //     before the MMAs read them (a NaN there would poison P.V even at P = 0).
 //   * Every wait is bounded; a wait that runs out sets the CTA's abort flag and
@@ -50,64 +50,72 @@ namespace {
 
 using namespace ptx;
 
-// warp 0 TMA, 1 QK^T issue, 2 PV issue, 3 length checks, 4-19 softmax (token
-// slice j = (warp - 4) / 4, lane quarter q = warp % 4), 20-23 query loaders
-constexpr int kBrSlices = 4;                          // 16-token slices of a page
-constexpr int kBrSliceTok = 64 / kBrSlices;
+// warp 0 TMA, 1 QK^T issue, 2 PV issue (and the length checks), 3-18 softmax:
+// token quarter jq = (warp - 3) / 4 of the unit (tokens 32 jq .. 32 jq + 31),
+// lane quarter q = warp % 4 (a warp reaches only the TMEM lanes of quarter
+// warp % 4); the warps with jq = 0 also load the query.
+constexpr int kBrUnitPages = 2;                 // pages of a unit (128 tokens)
+constexpr int kBrSlices = 4;                    // 32-token slices of a unit
 constexpr int kBrSmxWarps = 4 * kBrSlices;
-constexpr int kBrQWarp0 = 4 + kBrSmxWarps;
-constexpr int kBrThreads = 32 * (kBrQWarp0 + 4);
-constexpr int kBrSB = 4;                  // S buffers
-constexpr int kBrSlot = 64 * 128;         // 64 tokens x 64 bf16, 128-byte swizzle
-constexpr int kBrStage = 3 * kBrSlot;     // two latent blocks and the rope block of a page: 24 KB
-constexpr int kBrMaxStages = 9;
+constexpr int kBrSmxWarp0 = 3;
+constexpr int kBrThreads = 32 * (kBrSmxWarp0 + kBrSmxWarps);
+constexpr int kBrSB = 2;                        // S buffers: unit u uses u % 2
+constexpr int kBrSlot = 64 * 128;               // one page of one 64-dim block: 64 tokens x 64 bf16, 128-byte swizzle
+constexpr int kBrUnitSlot = 2 * kBrSlot;        // the same block of a unit's two pages, adjacent: 128 rows
+constexpr int kBrMaxUnits = 4;
 constexpr uint32_t kBrTmemCols = 512;
-// TMEM columns: O (128 latent dims), the S ring, the branch's query (128 bf16
-// = 64 packed columns) and the rope query (64 bf16 = 32 columns)
+// TMEM columns: O (128 latent dims), two S buffers (128 tokens each), the
+// query (128 bf16 = 64 packed columns) and the rope query (64 bf16 = 32)
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 128;
-constexpr uint32_t kColQ = kColS + 64 * kBrSB;
+constexpr uint32_t kColQ = kColS + 128 * kBrSB;
 constexpr uint32_t kColQR = kColQ + 64;
 static_assert(kColQR + 32 <= kBrTmemCols, "TMEM columns");
 
 struct BrBars {
-  uint64_t stage_full[kBrMaxStages], stage_empty[kBrMaxStages];
+  uint64_t unit_full[kBrMaxUnits], unit_empty[kBrMaxUnits];
   uint64_t s_full[kBrSB], p_full[kBrSB], pv_done[kBrSB];
   uint64_t q_full, q_empty, o_free;
-  uint64_t red_full[2][4], l_full[4];  // per lane quarter: its slice warps meet
-  float red[2][kBrSlices][128];        // [page parity][slice][head] maxima
-  float lsum[kBrSlices][128];          // [slice][head] softmax sums at the end of a piece
+  uint64_t red_full[4][2];  // per lane quarter, double-buffered: its four slices meet
+  uint64_t l_full[4];       // per lane quarter, at the end of a piece
+  float red[2][kBrSlices][128];  // [buffer][slice][head] maxima
+  float lsum[kBrSlices][128];    // [slice][head] sums at the end of a piece
   WorkerPlan plan;
   int page_ids[kIdRing];
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// Shared memory: the unit ring, block-major: block s (latent 0-63, latent
+// 64-127, rope) of ring entry k, page j at s * kBlockStride + k * kBrUnitSlot
+// + j * kBrSlot, so that a unit's two pages of a block are one 128-row operand.
 struct BrLayout {
   static constexpr int kCap = 232448;
   static constexpr int kTile = 0;
   static constexpr int kFixed = (int)sizeof(BrBars) + 1024;  // + alignment slack
-  static constexpr int kStages = (kCap - kFixed) / kBrStage < kBrMaxStages ? (kCap - kFixed) / kBrStage
-                                                                          : kBrMaxStages;
-  static constexpr int kBars = kTile + kStages * kBrStage;
+  static constexpr int kUnits = (kCap - kFixed) / (3 * kBrUnitSlot) < kBrMaxUnits ? (kCap - kFixed) / (3 * kBrUnitSlot)
+                                                                                   : kBrMaxUnits;
+  static constexpr int kBlockStride = kUnits * kBrUnitSlot;
+  static constexpr int kBars = kTile + 3 * kBlockStride;
   static constexpr int kBytes = kBars + (int)sizeof(BrBars) + 1024;
-  static_assert(kBrStage % 1024 == 0, "swizzle atoms stay aligned");
-  static_assert(kStages >= 4 && kBytes <= kCap, "shared memory");
+  static_assert(kBrUnitSlot % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(kUnits == kBrMaxUnits && kBytes <= kCap, "shared memory");
+  static_assert((kBlockStride >> 4) < (1 << 14), "the block stride fits the descriptor's leading byte offset");
 };
 
 // Optional pipeline trace (builds with -DMLRA_TRACE only): globaltimer stamps
-// of each role's events for the first kBrTracePages pages of CTAs 0 and 1.
+// of each role's events for the first kBrTraceUnits units of CTAs 0 and 1.
 #ifdef MLRA_TRACE
-constexpr int kBrTracePages = 64;
-__device__ unsigned long long g_btrace[2][kBrTracePages][16];
+constexpr int kBrTraceUnits = 64;
+__device__ unsigned long long g_btrace[2][kBrTraceUnits][16];
 enum { kTbTma = 0, kTbStageSeen, kTbQkIssued, kTbSLoaded, kTbRedDone, kTbPReady, kTbPSeen, kTbPvIssued,
        kTbStageFree, kTbSLoaded1, kTbPReady1 };
-#define BR_TRACE(gg, ev)                                                                                   \
+#define BR_TRACE(uu, ev)                                                                                   \
   do {                                                                                                     \
-    if (blockIdx.x < 2 && (gg) < (uint32_t)kBrTracePages) g_btrace[blockIdx.x][gg][ev] = globaltimer_ns(); \
+    if (blockIdx.x < 2 && (uu) < (uint32_t)kBrTraceUnits) g_btrace[blockIdx.x][uu][ev] = globaltimer_ns(); \
   } while (0)
 #else
-#define BR_TRACE(gg, ev) \
+#define BR_TRACE(uu, ev) \
   do {                   \
   } while (0)
 #endif
@@ -115,21 +123,43 @@ enum { kTbTma = 0, kTbStageSeen, kTbQkIssued, kTbSLoaded, kTbRedDone, kTbPReady,
 enum { kSiteQEmpty = 1, kSiteStageEmpty, kSiteQFull, kSiteMma, kSiteOFree, kSiteSFull, kSitePFull, kSitePvDone,
        kSiteRed, kSiteL };
 
+// The units of a piece: pages [pg0, pg1) of the piece in pairs, numbered
+// globally from u0.
+struct UnitRange {
+  uint32_t u0, u_end;
+  int pg0, pg1, L;
+  __device__ __forceinline__ int first_page(uint32_t u) const { return pg0 + kBrUnitPages * (int)(u - u0); }
+  __device__ __forceinline__ int pages(uint32_t u) const { return min(kBrUnitPages, pg1 - first_page(u)); }
+  // tokens of the unit inside the sequence (a piece may end before the sequence does)
+  __device__ __forceinline__ int valid(uint32_t u) const { return min(pages(u) * kPage, L - first_page(u) * kPage); }
+};
+__device__ __forceinline__ UnitRange units_of(const SegWalk& w, uint32_t u0) {
+  UnitRange r;
+  r.u0 = u0;
+  r.u_end = u0 + (uint32_t)((w.pg1 - w.pg0 + kBrUnitPages - 1) / kBrUnitPages);
+  r.pg0 = w.pg0;
+  r.pg1 = w.pg1;
+  r.L = w.L;
+  return r;
+}
+
 __global__ void __launch_bounds__(kBrThreads, 1)
     attend_tc_branch_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
                             const __nv_bfloat16* __restrict__ q_ws, const int* __restrict__ page_table,
                             const int* __restrict__ seq_lens, float* __restrict__ o_part,
                             float* __restrict__ ml_part, int* __restrict__ err, AttnArgs a) {
   using L = BrLayout;
-  constexpr int kStages = L::kStages;
-  constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);  // B = page latent read MN-major
+  constexpr int kUnits = L::kUnits;
+  constexpr uint32_t kIdescQK1 = idesc_bf16_f32(128, 64, false, false);   // one page
+  constexpr uint32_t kIdescQK2 = idesc_bf16_f32(128, 128, false, false);  // two pages
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);    // B = the latent read MN-major
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sTile = smem + L::kTile;
   BrBars* bars = reinterpret_cast<BrBars*>(smem + L::kBars);
   volatile int* abort_flag = &bars->abort_flag;
+  auto block_of = [&](int s2, uint32_t k, int j) { return sTile + s2 * L::kBlockStride + k * kBrUnitSlot + j * kBrSlot; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dep_launch();  // the combine kernel may set up (and load its weights) as this grid retires
@@ -139,21 +169,21 @@ __global__ void __launch_bounds__(kBrThreads, 1)
   const int d_cb = a.d_c / a.n_branch;  // 128
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&bars->stage_full[s]), 1);
-      mbar_init(smem_u32(&bars->stage_empty[s]), 1);
+    for (int k = 0; k < kUnits; ++k) {
+      mbar_init(smem_u32(&bars->unit_full[k]), 1);
+      mbar_init(smem_u32(&bars->unit_empty[k]), 1);
     }
     for (int k = 0; k < kBrSB; ++k) {
       mbar_init(smem_u32(&bars->s_full[k]), 1);
-      mbar_init(smem_u32(&bars->p_full[k]), kBrSmxWarps);  // every slice of every lane quarter
+      mbar_init(smem_u32(&bars->p_full[k]), kBrSmxWarps);
       mbar_init(smem_u32(&bars->pv_done[k]), 1);
     }
-    mbar_init(smem_u32(&bars->q_full), 4);
+    mbar_init(smem_u32(&bars->q_full), 4);  // the query loaders, one per lane quarter
     mbar_init(smem_u32(&bars->q_empty), 1);
     mbar_init(smem_u32(&bars->o_free), kBrSmxWarps);
     for (int q = 0; q < 4; ++q) {
-      mbar_init(smem_u32(&bars->red_full[0][q]), kBrSlices);
-      mbar_init(smem_u32(&bars->red_full[1][q]), kBrSlices);
+      mbar_init(smem_u32(&bars->red_full[q][0]), kBrSlices);
+      mbar_init(smem_u32(&bars->red_full[q][1]), kBrSlices);
       mbar_init(smem_u32(&bars->l_full[q]), kBrSlices);
     }
     bars->abort_flag = 0;
@@ -167,7 +197,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     WorkerPlan p = plan_worker(seq_lens, a.B, a.G, c, maxL);
     if (lane == 0) bars->plan = p;
   }
-  if (warp == 3 && blockIdx.x == 0) {
+  if (warp == 2 && blockIdx.x == 0) {
     for (int b = lane; b < a.B; b += 32) {
       const int Lb = __ldg(seq_lens + b);
       if (Lb < 0 || Lb > maxL) report_error(err, kErrDeviceCheck, b, Lb);
@@ -181,7 +211,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
-    // Pages stream through the stage ring in walk order, across pieces (the
+    // The pages through the unit ring in walk order, across pieces (the
     // cache does not depend on the query).  Page ids are read kIdAhead pages
     // before their tile and parked in a small ring.
     IdFetch ids(plan, a.B, maxL, seq_lens);
@@ -202,220 +232,232 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       tma_prefetch_desc(&tm_rope);
       SegWalk walk(plan, a.B, maxL);
       int* id_ring = bars->page_ids;
-      int pend = 0;
-      bool has_pend = false;
-      uint32_t g = 0;
+      // ids fetched while the previous unit was issued (pages pend_g, pend_g + 1), parked in the ring at
+      // the next unit, so that a page-table load never sits between a freed ring entry and its refill
+      int pend0 = 0, pend1 = 0, npend = 0;
+      uint32_t pend_g = 0;
+      uint32_t g = 0, u_next = 0;
       bool ok = true;
       while (ok && walk.next(seq_lens)) {
-        for (int p = walk.pg0; p < walk.pg1; ++p, ++g) {
-          if (has_pend) id_ring[(g - 1 + kIdAhead) % kIdRing] = pend;
-          has_pend = ids.live;
-          if (has_pend) pend = ids.fetch(seq_lens, page_table, a.maxp);  // the id of page g + kIdAhead
-          const uint32_t st = g % kStages, use = g / kStages;
-          if (use > 0 && !mbar_wait(smem_u32(&bars->stage_empty[st]), (use - 1) & 1, abort_flag, err,
-                                    kSiteStageEmpty)) {
+        const UnitRange ur = units_of(walk, u_next);
+        for (uint32_t u = ur.u0; ok && u < ur.u_end; ++u) {
+          const uint32_t k = u % kUnits, use = u / kUnits;
+          if (use > 0 && !mbar_wait(smem_u32(&bars->unit_empty[k]), (use - 1) & 1, abort_flag, err, kSiteStageEmpty)) {
             ok = false;
             break;
           }
-          BR_TRACE(g, kTbStageFree);
-          int pg = id_ring[g % kIdRing];
-          if (pg < 0 || pg >= a.num_pages) {  // reported, and replaced by page 0 so that no load leaves the pool
-            report_error(err, kErrDeviceCheck, walk.b, p * kPage);
-            pg = 0;
+          BR_TRACE(u, kTbStageFree);
+          const int np = ur.pages(u);
+          if (npend > 0) id_ring[pend_g % kIdRing] = pend0;
+          if (npend > 1) id_ring[(pend_g + 1) % kIdRing] = pend1;
+          npend = 0;
+          pend_g = g + kIdAhead;
+          static_assert(kBrUnitPages == 2, "two ids in flight per unit");
+          if (ids.live) {  // the ids of pages g + kIdAhead (+ 1), in flight until the next unit
+            pend0 = ids.fetch(seq_lens, page_table, a.maxp);
+            npend = 1;
+            if (np > 1 && ids.live) {
+              pend1 = ids.fetch(seq_lens, page_table, a.maxp);
+              npend = 2;
+            }
           }
-          const uint32_t fb = smem_u32(&bars->stage_full[st]);
-          uint8_t* tile = sTile + st * kBrStage;
-          mbar_expect_tx(fb, kBrStage);
-          tma_load_2d(smem_u32(tile), &tm_lat, fb, d_cb * br, pg * kPage);
-          tma_load_2d(smem_u32(tile + kBrSlot), &tm_lat, fb, d_cb * br + 64, pg * kPage);
-          tma_load_2d(smem_u32(tile + 2 * kBrSlot), &tm_rope, fb, 0, pg * kPage);
-          BR_TRACE(g, kTbTma);
+          const uint32_t fb = smem_u32(&bars->unit_full[k]);
+          mbar_expect_tx(fb, (uint32_t)(np * 3 * kBrSlot));
+          for (int j = 0; j < np; ++j, ++g) {
+            int pg = id_ring[g % kIdRing];
+            if (pg < 0 || pg >= a.num_pages) {  // reported, and replaced by page 0 so that no load leaves the pool
+              report_error(err, kErrDeviceCheck, walk.b, (ur.first_page(u) + j) * kPage);
+              pg = 0;
+            }
+            tma_load_2d(smem_u32(block_of(0, k, j)), &tm_lat, fb, d_cb * br, pg * kPage);
+            tma_load_2d(smem_u32(block_of(1, k, j)), &tm_lat, fb, d_cb * br + 64, pg * kPage);
+            tma_load_2d(smem_u32(block_of(2, k, j)), &tm_rope, fb, 0, pg * kPage);
+          }
+          BR_TRACE(u, kTbTma);
         }
+        u_next = ur.u_end;
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------------- QK^T
-    // QK^T of every page in walk order, as soon as it has landed and PV has
-    // consumed the P written over its S buffer (which implies both softmax
-    // halves have read the scores it held).
+    // QK^T a unit at a time (one N = 128 MMA per 16 dims for two pages), as
+    // soon as the unit has landed and PV has consumed the P written over its S
+    // buffer (which implies the softmax has read the scores it held).
     SegWalk walk(plan, a.B, maxL);
     int seg = 0;
-    uint32_t g = 0;
+    uint32_t u_next = 0;
     bool ok = true;
     while (ok && walk.next(seq_lens)) {
       if (!mbar_wait_warp(smem_u32(&bars->q_full), seg & 1, abort_flag, err, kSiteQFull)) break;
       tc_fence_after();
-      const uint32_t g0 = g, g_end = g + (uint32_t)(walk.pg1 - walk.pg0);
-      for (; g < g_end; ++g) {
-        const uint32_t st = g % kStages;
-        // S buffer g % kBrSB holds P(g - kBrSB) until PV(g - kBrSB) has completed
-        if (!mbar_wait_warp(smem_u32(&bars->stage_full[st]), (g / kStages) & 1, abort_flag, err, kSiteMma) ||
-            (g >= (uint32_t)kBrSB && !mbar_wait_warp(smem_u32(&bars->pv_done[g % kBrSB]), ((g / kBrSB) - 1) & 1,
+      const UnitRange ur = units_of(walk, u_next);
+      for (uint32_t u = ur.u0; u < ur.u_end; ++u) {
+        const uint32_t k = u % kUnits;
+        if (!mbar_wait_warp(smem_u32(&bars->unit_full[k]), (u / kUnits) & 1, abort_flag, err, kSiteMma) ||
+            (u >= (uint32_t)kBrSB && !mbar_wait_warp(smem_u32(&bars->pv_done[u % kBrSB]), ((u / kBrSB) - 1) & 1,
                                                       abort_flag, err, kSitePvDone))) {
           ok = false;
           break;
         }
-        if (lane == 0) BR_TRACE(g, kTbStageSeen);
-        uint8_t* tile = sTile + st * kBrStage;
-        const int p = walk.pg0 + (int)(g - g0);
-        const int valid = min(kPage, walk.L - p * kPage);
-        if (valid < kPage) {  // zero the rows past the end of the sequence (both latent blocks, rope block)
-          const int nrow = kPage - valid;
+        if (lane == 0) BR_TRACE(u, kTbStageSeen);
+        const int np = ur.pages(u);
+        const int valid = ur.valid(u);
+        if (valid < np * kPage) {  // zero the rows past the end of the sequence in the unit's last page
+          const int j = np - 1, v = valid - j * kPage, nrow = kPage - v;
           const uint4 z = make_uint4(0, 0, 0, 0);
           for (int idx = lane; idx < nrow * 8 * 3; idx += 32) {
             const int s2 = idx / (nrow * 8), rem = idx % (nrow * 8);
-            *reinterpret_cast<uint4*>(tile + s2 * kBrSlot + (valid + rem / 8) * 128 + (rem % 8) * 16) = z;
+            *reinterpret_cast<uint4*>(block_of(s2, k, j) + (v + rem / 8) * 128 + (rem % 8) * 16) = z;
           }
           fence_proxy_async_smem();
         }
         __syncwarp();
         tc_fence_after();
         if (lane == 0) {
-          const uint64_t td = sdesc_sw128(smem_u32(tile), 16, 1024);
-          const uint32_t s_col = tmem + kColS + (g % kBrSB) * 64u;
+          const uint64_t td = sdesc_sw128(smem_u32(block_of(0, k, 0)), 16, 1024);
+          const uint32_t s_col = tmem + kColS + (u % kBrSB) * 128u;
+          const uint32_t idesc = np == 2 ? kIdescQK2 : kIdescQK1;
 #pragma unroll
           for (int s2 = 0; s2 < 2; ++s2)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-              mma_ts(s_col, tmem + kColQ + 32u * s2 + 8u * ks, td + (uint64_t)((s2 * kBrSlot + ks * 32) >> 4),
-                     kIdescQK, (s2 | ks) ? 1u : 0u);
+              mma_ts(s_col, tmem + kColQ + 32u * s2 + 8u * ks, td + (uint64_t)((s2 * L::kBlockStride + ks * 32) >> 4),
+                     idesc, (s2 | ks) ? 1u : 0u);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(s_col, tmem + kColQR + 8u * ks, td + (uint64_t)((2 * kBrSlot + ks * 32) >> 4), kIdescQK, 1u);
-          mma_commit(smem_u32(&bars->s_full[g % kBrSB]));
-          if (g + 1 == g_end) mma_commit(smem_u32(&bars->q_empty));  // the last read of this query
-          BR_TRACE(g, kTbQkIssued);
+            mma_ts(s_col, tmem + kColQR + 8u * ks, td + (uint64_t)((2 * L::kBlockStride + ks * 32) >> 4), idesc, 1u);
+          mma_commit(smem_u32(&bars->s_full[u % kBrSB]));
+          if (u + 1 == ur.u_end) mma_commit(smem_u32(&bars->q_empty));  // the last read of this query
+          BR_TRACE(u, kTbQkIssued);
         }
         __syncwarp();
       }
+      u_next = ur.u_end;
       ++seg;
     }
   } else if (warp == 2) {
     // ----------------------------------------------------------------- PV
-    // PV of every page in walk order, as soon as every slice of its P is in
-    // TMEM; the commits free the page's stage and its S buffer.
+    // PV a unit at a time into O, as soon as every slice of its P is in
+    // TMEM; the commits free the unit's ring entry and its S buffer.
     SegWalk walk(plan, a.B, maxL);
     int seg = 0;
-    uint32_t g = 0;
+    uint32_t u_next = 0;
     bool ok = true;
     while (ok && walk.next(seq_lens)) {
       // the previous piece's O must be read out before the first PV overwrites it
       if (seg > 0 && !mbar_wait_warp(smem_u32(&bars->o_free), (seg - 1) & 1, abort_flag, err, kSiteOFree)) break;
-      const uint32_t g0 = g, g_end = g + (uint32_t)(walk.pg1 - walk.pg0);
-      for (; g < g_end; ++g) {
-        if (!mbar_wait_warp(smem_u32(&bars->p_full[g % kBrSB]), (g / kBrSB) & 1, abort_flag, err, kSitePFull)) {
+      const UnitRange ur = units_of(walk, u_next);
+      for (uint32_t u = ur.u0; u < ur.u_end; ++u) {
+        if (!mbar_wait_warp(smem_u32(&bars->p_full[u % kBrSB]), (u / kBrSB) & 1, abort_flag, err, kSitePFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          BR_TRACE(g, kTbPSeen);
-          const uint32_t first = g == g0 ? 1u : 0u;
-          const uint64_t vd = sdesc_sw128(smem_u32(sTile + (g % kStages) * kBrStage), 8192, 1024);
-          const uint32_t p_base = tmem + kColS + (g % kBrSB) * 64u;
+          BR_TRACE(u, kTbPSeen);
+          const uint32_t k = u % kUnits;
+          const uint64_t vd = sdesc_sw128(smem_u32(block_of(0, k, 0)), (uint32_t)L::kBlockStride, 1024);
+          const uint32_t p_base = tmem + kColS + (u % kBrSB) * 128u;
+          // P of tokens 16 ks .. 16 ks + 15 (slice ks / 2): packed columns 32 (ks / 2) + 16 + 8 (ks % 2)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tmem + kColO, p_base + 8u * ks, vd + (uint64_t)((ks * 2048) >> 4), kIdescPV,
-                   ks == 0 ? (first ^ 1u) : 1u);
-          mma_commit(smem_u32(&bars->stage_empty[g % kStages]));
-          mma_commit(smem_u32(&bars->pv_done[g % kBrSB]));
-          BR_TRACE(g, kTbPvIssued);
+            mma_ts(tmem + kColO, p_base + 32u * (ks >> 1) + 16u + 8u * (ks & 1), vd + (uint64_t)((ks * 2048) >> 4),
+                   kIdescPV, (u == ur.u0 && ks == 0) ? 0u : 1u);
+          if (ur.pages(u) == 2) {
+#pragma unroll
+            for (int ks = 4; ks < 8; ++ks)
+              mma_ts(tmem + kColO, p_base + 32u * (ks >> 1) + 16u + 8u * (ks & 1), vd + (uint64_t)((ks * 2048) >> 4),
+                     kIdescPV, 1u);
+          }
+          mma_commit(smem_u32(&bars->unit_empty[k]));
+          mma_commit(smem_u32(&bars->pv_done[u % kBrSB]));
+          BR_TRACE(u, kTbPvIssued);
         }
         __syncwarp();
       }
+      u_next = ur.u_end;
       ++seg;
     }
-  } else if (warp >= kBrQWarp0) {
-    // -------------------------------------------------------------- query
-    // Quarter q: the query rows of heads 32q + lane (this branch's 128 latent
-    // dims as 64 packed bf16x2 columns, the 64 rope dims as 32) into TMEM for
-    // each piece, once the previous piece's last QK^T has completed.
-    const int q = warp & 3;
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const int head = q * 32 + lane;
-    const bool real = head < a.H;
-    grid_dep_wait();  // the absorbed queries come from the previous kernel
-    SegWalk walk(plan, a.B, maxL);
-    int seg = 0;
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    while (walk.next(seq_lens)) {
-      if (seg > 0 && !mbar_wait_warp(smem_u32(&bars->q_empty), (seg - 1) & 1, abort_flag, err, kSiteQEmpty)) break;
-      tc_fence_after();
-      const __nv_bfloat16* src = q_ws + ((size_t)walk.b * a.H + (real ? head : 0)) * (a.d_c + a.d_r);
-      const uint4* lat = reinterpret_cast<const uint4*>(src + d_cb * br);
-      const uint4* rop = reinterpret_cast<const uint4*>(src + a.d_c);
-#pragma unroll
-      for (int blk = 0; blk < 3; ++blk) {  // latent columns 0-31, 32-63, then the rope's 32
-        const uint4* from = blk < 2 ? lat + 8 * blk : rop;
-        uint32_t r[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = real ? __ldg(from + i) : z;
-          r[4 * i] = v.x;
-          r[4 * i + 1] = v.y;
-          r[4 * i + 2] = v.z;
-          r[4 * i + 3] = v.w;
-        }
-        tmem_st32(tmem + lane_off + (blk < 2 ? kColQ + 32u * blk : kColQR), r);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
-      ++seg;
-    }
-  } else if (warp >= 4) {
+  } else if (warp >= kBrSmxWarp0) {
     // -------------------------------------------------------------- softmax
-    // Lane quarter q (heads 32q + lane), token slice j of each page.
+    // Lane quarter q (heads 32q + lane), token slice jq of each unit.
+    const int sw = warp - kBrSmxWarp0;
+    const int jq = sw / 4;
     const int q = warp & 3;
-    const int j = (warp - 4) >> 2;
     const int head = q * 32 + lane;
     const bool real = head < a.H;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     SegWalk walk(plan, a.B, maxL);
-    uint32_t g = 0;
+    uint32_t u_next = 0;
     int seg = 0;
     bool ok = true;
+    if (jq == 0) grid_dep_wait();  // the absorbed queries come from the previous kernel
     while (ok && walk.next(seq_lens)) {
-      const uint32_t g0 = g, g_end = g + (uint32_t)(walk.pg1 - walk.pg0);
+      if (jq == 0) {
+        // the piece's query rows of heads 32q + lane (this branch's 128 latent dims as 64 packed bf16x2
+        // columns, the 64 rope dims as 32) into TMEM, once the previous piece's last QK^T has completed
+        if (seg > 0 && !mbar_wait_warp(smem_u32(&bars->q_empty), (seg - 1) & 1, abort_flag, err, kSiteQEmpty)) break;
+        tc_fence_after();
+        const __nv_bfloat16* src = q_ws + ((size_t)walk.b * a.H + (real ? head : 0)) * (a.d_c + a.d_r);
+        const uint4* lat = reinterpret_cast<const uint4*>(src + d_cb * br);
+        const uint4* rop = reinterpret_cast<const uint4*>(src + a.d_c);
+        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int blk = 0; blk < 3; ++blk) {  // latent columns 0-31, 32-63, then the rope's 32
+          const uint4* from = blk < 2 ? lat + 8 * blk : rop;
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 v = real ? __ldg(from + i) : z;
+            r[4 * i] = v.x;
+            r[4 * i + 1] = v.y;
+            r[4 * i + 2] = v.z;
+            r[4 * i + 3] = v.w;
+          }
+          tmem_st32(tmem + lane_off + (blk < 2 ? kColQ + 32u * blk : kColQR), r);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
+      }
+      const UnitRange ur = units_of(walk, u_next);
       float m_run = -INFINITY, l_run = 0.f;
-      for (; g < g_end; ++g) {
-        const int valid = min(kPage, walk.L - (walk.pg0 + (int)(g - g0)) * kPage);
-        const uint32_t s_col = kColS + (g % kBrSB) * 64u;
-        if (!mbar_wait_warp(smem_u32(&bars->s_full[g % kBrSB]), (g / kBrSB) & 1, abort_flag, err, kSiteSFull)) {
+      for (uint32_t u = ur.u0; u < ur.u_end; ++u) {
+        const int valid = ur.valid(u) - 32 * jq;  // valid tokens of this slice (<= 0: none)
+        // scores of token 32 jq + t at column s_sl + t; its P (bf16) at packed column s_sl + 16 + t / 2
+        const uint32_t s_sl = tmem + lane_off + kColS + (u % kBrSB) * 128u + 32u * (uint32_t)jq;
+        if (!mbar_wait_warp(smem_u32(&bars->s_full[u % kBrSB]), (u / kBrSB) & 1, abort_flag, err, kSiteSFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float s[kBrSliceTok];
-        {
-          uint32_t v[16];
-          tmem_ld16(tmem + lane_off + s_col + (uint32_t)(kBrSliceTok * j), v);
-#pragma unroll
-          for (int i = 0; i < kBrSliceTok; ++i)
-            s[i] = kBrSliceTok * j + i < valid ? __uint_as_float(v[i]) : -INFINITY;
-        }
-        if (q == 0 && lane == 0 && j < 2) BR_TRACE(g, j == 0 ? kTbSLoaded : kTbSLoaded1);
-        tc_fence_before();  // the scores are read before the barrier below lets the other slices write P
+        uint32_t vhi[16], vlo[16];
+        tmem_ld16(s_sl + 16u, vhi);  // tokens 16-31 of the slice (their columns take the P)
+        tmem_ld16(s_sl, vlo);        // tokens 0-15
         float m4[4];
 #pragma unroll
-        for (int i = 0; i < kBrSliceTok; ++i) m4[i & 3] = i < 4 ? s[i] : fmaxf(m4[i & 3], s[i]);
-        const int buf = g & 1;
-        bars->red[buf][j][head] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        for (int i = 0; i < 16; ++i) {
+          const float x = i < valid ? __uint_as_float(vlo[i]) : -INFINITY;
+          const float y = 16 + i < valid ? __uint_as_float(vhi[i]) : -INFINITY;
+          m4[i & 3] = i < 4 ? fmaxf(x, y) : fmaxf(m4[i & 3], fmaxf(x, y));
+        }
+        if (q == 0 && lane == 0) BR_TRACE(u, jq == 0 ? kTbSLoaded : kTbSLoaded1);
+        const int rb = (int)(u & 1u);
+        bars->red[rb][jq][head] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->red_full[buf][q]));
-        if (!mbar_wait_warp(smem_u32(&bars->red_full[buf][q]), (g >> 1) & 1, abort_flag, err, kSiteRed)) {
+        if (lane == 0) mbar_arrive(smem_u32(&bars->red_full[q][rb]));
+        if (!mbar_wait_warp(smem_u32(&bars->red_full[q][rb]), (u >> 1) & 1, abort_flag, err, kSiteRed)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (q == 0 && j == 0 && lane == 0) BR_TRACE(g, kTbRedDone);
-        // the page's row maximum (at least one token of a page is valid, so it is finite); the slices
-        // of a quarter read the same four values and decide alike
-        const float M = fmaxf(fmaxf(bars->red[buf][0][head], bars->red[buf][1][head]),
-                              fmaxf(bars->red[buf][2][head], bars->red[buf][3][head]));
+        if (q == 0 && jq == 0 && lane == 0) BR_TRACE(u, kTbRedDone);
+        // the unit's row maximum (its first token is valid, so it is finite); the four slices of a quarter
+        // read the same four values and decide alike
+        const float M = fmaxf(fmaxf(bars->red[rb][0][head], bars->red[rb][1][head]),
+                              fmaxf(bars->red[rb][2][head], bars->red[rb][3][head]));
         float m_use, corr;
         bool rescale = false;
-        if (g == g0) {
+        if (u == ur.u0) {
           m_use = M;
           corr = 0.f;
         } else if (M > m_run + kRescaleLog2) {
@@ -426,63 +468,73 @@ __global__ void __launch_bounds__(kBrThreads, 1)
           m_use = m_run;
           corr = 1.f;
         }
+        uint32_t pk[16];
         float a4[4];
 #pragma unroll
-        for (int i = 0; i < kBrSliceTok; ++i) {
-          s[i] = ex2(s[i] - m_use);
-          a4[i & 3] = i < 4 ? s[i] : a4[i & 3] + s[i];
+        for (int i = 0; i < 8; ++i) {
+          const float p0 = 2 * i < valid ? ex2(__uint_as_float(vlo[2 * i]) - m_use) : 0.f;
+          const float p1 = 2 * i + 1 < valid ? ex2(__uint_as_float(vlo[2 * i + 1]) - m_use) : 0.f;
+          const float p2 = 16 + 2 * i < valid ? ex2(__uint_as_float(vhi[2 * i]) - m_use) : 0.f;
+          const float p3 = 17 + 2 * i < valid ? ex2(__uint_as_float(vhi[2 * i + 1]) - m_use) : 0.f;
+          a4[0] = i == 0 ? p0 : a4[0] + p0;
+          a4[1] = i == 0 ? p1 : a4[1] + p1;
+          a4[2] = i == 0 ? p2 : a4[2] + p2;
+          a4[3] = i == 0 ? p3 : a4[3] + p3;
+          pk[i] = pack_bf16x2(p0, p1);
+          pk[8 + i] = pack_bf16x2(p2, p3);
         }
+        tmem_st16(s_sl + 16u, pk);  // over the scores of tokens 16-31, read above
         l_run = l_run * corr + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
         m_run = m_use;
-        // O is rescaled only when the running max jumped; slice j takes columns [32j, 32j + 32)
+        // O is rescaled only when the running max jumped; slice jq takes columns [32 jq, 32 jq + 32)
         if (__any_sync(0xffffffffu, rescale)) {
-          if (!mbar_wait_warp(smem_u32(&bars->pv_done[(g - 1) % kBrSB]), ((g - 1) / kBrSB) & 1, abort_flag, err,
-                              kSitePvDone)) {
+          const uint32_t up = u - 1;  // the previous unit, in this piece since u != u0
+          if (!mbar_wait_warp(smem_u32(&bars->pv_done[up % kBrSB]), (up / kBrSB) & 1, abort_flag, err, kSitePvDone)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_off + kColO + 32u * j, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-          tmem_st32(tmem + lane_off + kColO + 32u * j, o);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t o[16];
+            const uint32_t col = tmem + lane_off + kColO + 32u * (uint32_t)jq + 16u * h2;
+            tmem_ld16(col, o);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+            tmem_st16(col, o);
+          }
         }
-        // P (bf16) over the S buffer: slice j's 16 tokens are packed columns [8j, 8j + 8).  Every slice
-        // loaded its scores before any passed the barrier above, so nothing unread is overwritten.
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        tmem_st8(tmem + lane_off + s_col + 8u * j, pk);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[g % kBrSB]));
-        if (q == 0 && lane == 0 && j < 2) BR_TRACE(g, j == 0 ? kTbPReady : kTbPReady1);
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[u % kBrSB]));
+        if (q == 0 && lane == 0) BR_TRACE(u, jq == 0 ? kTbPReady : kTbPReady1);
       }
       if (!ok) break;
-      // epilogue: slice j writes O columns [32j, 32j + 32) of its head; (m, l) of the piece
-      if (!mbar_wait_warp(smem_u32(&bars->pv_done[(g - 1) % kBrSB]), ((g - 1) / kBrSB) & 1, abort_flag, err,
-                          kSitePvDone))
+      // epilogue: slice jq writes O columns [32 jq, 32 jq + 32) of its head; (m, l) of the piece.  PV of the
+      // piece's last unit completing implies all of its PVs have (one issuing thread, completed in order).
+      const uint32_t last = ur.u_end - 1;
+      if (!mbar_wait_warp(smem_u32(&bars->pv_done[last % kBrSB]), (last / kBrSB) & 1, abort_flag, err, kSitePvDone))
         break;
       tc_fence_after();
       const int slot = c + walk.b;
-      {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_off + kColO + 32u * j, o);
-        if (real) {
-          float4* dst =
-              reinterpret_cast<float4*>(o_part + ((size_t)slot * a.H + head) * a.d_c + d_cb * br + 32 * j);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t o[16];
+        tmem_ld16(tmem + lane_off + kColO + 32u * (uint32_t)jq + 16u * h2, o);
+        if (real) {
+          float4* dst = reinterpret_cast<float4*>(o_part + ((size_t)slot * a.H + head) * a.d_c + d_cb * br + 32 * jq +
+                                                  16 * h2);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
             dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      bars->lsum[j][head] = l_run;
+      bars->lsum[jq][head] = l_run;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->l_full[q]));
       if (!mbar_wait_warp(smem_u32(&bars->l_full[q]), seg & 1, abort_flag, err, kSiteL)) break;
-      if (j == 0 && real) {
+      if (jq == 0 && real) {
         const float l = (bars->lsum[0][head] + bars->lsum[1][head]) + (bars->lsum[2][head] + bars->lsum[3][head]);
         ml_part[(((size_t)slot * a.n_branch + br) * 2 + 0) * a.H + head] = m_run;
         ml_part[(((size_t)slot * a.n_branch + br) * 2 + 1) * a.H + head] = l;
@@ -490,6 +542,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->o_free));
+      u_next = ur.u_end;
       ++seg;
     }
   }
@@ -511,13 +564,12 @@ extern "C" __attribute__((visibility("default"))) int mlra_branch_trace_read(uns
 }
 #endif
 
-// The kernel is written for n 128-dim branches, but the library sends it the
-// one-branch decode of a 128-dim latent only (the share of a branch-parallel
-// MLRA rank): MLRA-4 over a 512-dim latent ran faster on the four-CTA layout
-// of attn_tc.cu (202.8 against 234 us at 32 x 16384 tokens, 128 heads), whose
-// two CTAs per SM give two independent page pipelines.
+// Branches of 128 latent dims (MLRA over n_branch x 128 dims, and the
+// one-branch decode of a 128-dim latent that a branch-parallel MLRA rank runs),
+// 64 rope dims, 33 to 128 heads.
 bool tc_branch_supported(int H, int d_c, int d_r, int n_branch) {
-  return H > 32 && H <= 128 && d_r == 64 && n_branch == 1 && d_c == 128;
+  return H > 32 && H <= 128 && d_r == 64 && (n_branch == 1 || n_branch == 2 || n_branch == 4) &&
+         d_c == 128 * n_branch;
 }
 
 int tc_branch_workers(int sms, int n_branch) { return sms / n_branch > 0 ? sms / n_branch : 1; }

@@ -954,7 +954,10 @@ cudaError_t launch_attend_tc(const void* q_ws, const void* lat, const void* rop,
 }
 
 const char* tc_variant_name(int H, int d_c, int n_branch) {
-  if (tc_branch_supported(H, d_c, 64, n_branch)) return "attend_tc_branch_kernel<mla over a 128-dim latent>";
+  if (tc_branch_supported(H, d_c, 64, n_branch))
+    return n_branch == 1 ? "attend_tc_branch_kernel<mla over a 128-dim latent, two-page units>"
+                         : (n_branch == 2 ? "attend_tc_branch_kernel<mlra-2, one branch per cta, two-page units>"
+                                          : "attend_tc_branch_kernel<mlra-4, one branch per cta, two-page units>");
   const bool small = H <= 32;
   switch (n_branch) {
     case 1: return small ? "attend_tc_small_kernel<mla, cta pair, head-replicated query>"

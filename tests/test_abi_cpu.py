@@ -178,10 +178,11 @@ def test_describe_plan_follows_the_kernel_switch(L):
     d.kernel = 1
     assert abi.describe_plan(d)["family"] == "cuda-core"
     d.kernel = 2
-    assert abi.describe_plan(d)["attention"] == "attend_tc_kernel<mlra-4, four ctas, two per sm>"
-    # a branch-parallel rank's share (one 128-dim branch) runs on the branch kernel
+    assert abi.describe_plan(d)["attention"] == "attend_tc_branch_kernel<mlra-4, one branch per cta, two-page units>"
+    # MLRA-4 over 128-dim branches and a branch-parallel rank's share (one 128-dim branch) run on the
+    # branch kernel
     d1 = _workload_dims(w.with_(d_c=128, n_branch=1))
-    assert abi.describe_plan(d1)["attention"] == "attend_tc_branch_kernel<mla over a 128-dim latent>"
+    assert abi.describe_plan(d1)["attention"] == "attend_tc_branch_kernel<mla over a 128-dim latent, two-page units>"
     assert abi.describe_plan(d1)["family"] == "tcgen05"
     buf = ctypes.create_string_buffer(8)
     assert L.mlra_describe_plan(ctypes.byref(d), buf, len(buf)) == 1  # MLRA_ERR_INVALID_ARG
