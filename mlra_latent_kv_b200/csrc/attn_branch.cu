@@ -19,17 +19,21 @@
 //     a tcgen05 MMA of N <= 64 costs at least ~45 cycles whatever its size,
 //     and N = 128 runs at the full rate.  The unit is also the step of every
 //     barrier hand-off, which halves them against a page-sized step.
-//   * The branch's query (128 latent dims and 64 rope dims per head) lives in
-//     TMEM beside O (128 columns) and two S buffers of 128 columns, so shared
-//     memory holds only the unit ring: four units of 48 KB.
-//   * QK^T (M = 128 heads, N = 128 tokens, A = the query in TMEM) and PV (A =
-//     P in TMEM, B = the unit's latent read MN-major, N = 128 dims) are issued
-//     by two warps.
+//   * TMEM holds O (128 columns), two S buffers (128 each), one P buffer (64
+//     packed columns) and the branch's latent query (64 packed columns); the
+//     rope query (16 KB) sits in shared memory beside the unit ring (four
+//     units of 48 KB).  P has its own columns, so an S buffer is free again as
+//     soon as the softmax has read it: QK^T of unit u + 2 waits for that read,
+//     not for PV of unit u, and the softmax waits for PV of unit u - 1 only
+//     when it is about to store P.
+//   * QK^T (M = 128 heads, N = 128 tokens; the latent part with A = the query
+//     in TMEM, the rope part with A = the rope query in shared memory) and PV
+//     (A = P in TMEM, B = the unit's latent read MN-major, N = 128 dims) are
+//     issued by two warps.
 //   * Softmax: per TMEM lane quarter, four warps, one per 32 tokens of the
-//     unit; they agree on the unit's row maximum through shared memory, and
-//     each writes the P (bf16) of its tokens over its own score columns.  O is
+//     unit; they agree on the unit's row maximum through shared memory.  O is
 //     rescaled only when the running max grows by more than 2^8.  The first
-//     warp of each quarter also loads the query rows into TMEM per piece.
+//     warp of each quarter also loads the query rows per piece.
 //   * Rows past the sequence end in the last page are zeroed in shared memory
 //     before the MMAs read them (a NaN there would poison P.V even at P = 0).
 //   * Every wait is bounded; a wait that runs out sets the CTA's abort flag and
@@ -63,18 +67,22 @@ constexpr int kBrSB = 2;                        // S buffers: unit u uses u % 2
 constexpr int kBrSlot = 64 * 128;               // one page of one 64-dim block: 64 tokens x 64 bf16, 128-byte swizzle
 constexpr int kBrUnitSlot = 2 * kBrSlot;        // the same block of a unit's two pages, adjacent: 128 rows
 constexpr int kBrMaxUnits = 4;
+// Past a piece's first unit, scores are exponentiated against the running max before the unit's maximum
+// is known, capped at 2^64 (a sum of 128 such terms stays far inside fp32).
+constexpr float kSpecCapLog2 = 64.f;
 constexpr uint32_t kBrTmemCols = 512;
-// TMEM columns: O (128 latent dims), two S buffers (128 tokens each), the
-// query (128 bf16 = 64 packed columns) and the rope query (64 bf16 = 32)
+// TMEM columns: O (128 latent dims), two S buffers (128 tokens each), P (128
+// bf16 = 64 packed columns) and the latent query (128 bf16 = 64)
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 128;
-constexpr uint32_t kColQ = kColS + 128 * kBrSB;
-constexpr uint32_t kColQR = kColQ + 64;
-static_assert(kColQR + 32 <= kBrTmemCols, "TMEM columns");
+constexpr uint32_t kColP = kColS + 128 * kBrSB;
+constexpr uint32_t kColQ = kColP + 64;
+static_assert(kColQ + 64 <= kBrTmemCols, "TMEM columns");
+constexpr int kBrQRBytes = 128 * 128;  // rope query: 128 heads x 64 bf16, 128-byte swizzle
 
 struct BrBars {
   uint64_t unit_full[kBrMaxUnits], unit_empty[kBrMaxUnits];
-  uint64_t s_full[kBrSB], p_full[kBrSB], pv_done[kBrSB];
+  uint64_t s_full[kBrSB], s_free[kBrSB], p_full[kBrSB], pv_done[kBrSB];
   uint64_t q_full, q_empty, o_free;
   uint64_t red_full[4][2];  // per lane quarter, double-buffered: its four slices meet
   uint64_t l_full[4];       // per lane quarter, at the end of a piece
@@ -88,15 +96,17 @@ struct BrBars {
 
 // Shared memory: the unit ring, block-major: block s (latent 0-63, latent
 // 64-127, rope) of ring entry k, page j at s * kBlockStride + k * kBrUnitSlot
-// + j * kBrSlot, so that a unit's two pages of a block are one 128-row operand.
+// + j * kBrSlot, so that a unit's two pages of a block are one 128-row operand;
+// then the rope query.
 struct BrLayout {
   static constexpr int kCap = 232448;
   static constexpr int kTile = 0;
-  static constexpr int kFixed = (int)sizeof(BrBars) + 1024;  // + alignment slack
+  static constexpr int kFixed = kBrQRBytes + (int)sizeof(BrBars) + 1024;  // + alignment slack
   static constexpr int kUnits = (kCap - kFixed) / (3 * kBrUnitSlot) < kBrMaxUnits ? (kCap - kFixed) / (3 * kBrUnitSlot)
                                                                                    : kBrMaxUnits;
   static constexpr int kBlockStride = kUnits * kBrUnitSlot;
-  static constexpr int kBars = kTile + 3 * kBlockStride;
+  static constexpr int kQR = kTile + 3 * kBlockStride;
+  static constexpr int kBars = kQR + kBrQRBytes;
   static constexpr int kBytes = kBars + (int)sizeof(BrBars) + 1024;
   static_assert(kBrUnitSlot % 1024 == 0, "swizzle atoms stay aligned");
   static_assert(kUnits == kBrMaxUnits && kBytes <= kCap, "shared memory");
@@ -157,6 +167,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sTile = smem + L::kTile;
+  uint8_t* sQR = smem + L::kQR;
   BrBars* bars = reinterpret_cast<BrBars*>(smem + L::kBars);
   volatile int* abort_flag = &bars->abort_flag;
   auto block_of = [&](int s2, uint32_t k, int j) { return sTile + s2 * L::kBlockStride + k * kBrUnitSlot + j * kBrSlot; };
@@ -175,6 +186,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     }
     for (int k = 0; k < kBrSB; ++k) {
       mbar_init(smem_u32(&bars->s_full[k]), 1);
+      mbar_init(smem_u32(&bars->s_free[k]), kBrSmxWarps);
       mbar_init(smem_u32(&bars->p_full[k]), kBrSmxWarps);
       mbar_init(smem_u32(&bars->pv_done[k]), 1);
     }
@@ -281,8 +293,8 @@ __global__ void __launch_bounds__(kBrThreads, 1)
   } else if (warp == 1) {
     // --------------------------------------------------------------- QK^T
     // QK^T a unit at a time (one N = 128 MMA per 16 dims for two pages), as
-    // soon as the unit has landed and PV has consumed the P written over its S
-    // buffer (which implies the softmax has read the scores it held).
+    // soon as the unit has landed and the softmax has read the scores its S
+    // buffer held two units ago.
     SegWalk walk(plan, a.B, maxL);
     int seg = 0;
     uint32_t u_next = 0;
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       for (uint32_t u = ur.u0; u < ur.u_end; ++u) {
         const uint32_t k = u % kUnits;
         if (!mbar_wait_warp(smem_u32(&bars->unit_full[k]), (u / kUnits) & 1, abort_flag, err, kSiteMma) ||
-            (u >= (uint32_t)kBrSB && !mbar_wait_warp(smem_u32(&bars->pv_done[u % kBrSB]), ((u / kBrSB) - 1) & 1,
+            (u >= (uint32_t)kBrSB && !mbar_wait_warp(smem_u32(&bars->s_free[u % kBrSB]), ((u / kBrSB) - 1) & 1,
                                                       abort_flag, err, kSitePvDone))) {
           ok = false;
           break;
@@ -323,9 +335,11 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             for (int ks = 0; ks < 4; ++ks)
               mma_ts(s_col, tmem + kColQ + 32u * s2 + 8u * ks, td + (uint64_t)((s2 * L::kBlockStride + ks * 32) >> 4),
                      idesc, (s2 | ks) ? 1u : 0u);
+          const uint64_t qrd = sdesc_sw128(smem_u32(sQR), 16, 1024);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(s_col, tmem + kColQR + 8u * ks, td + (uint64_t)((2 * L::kBlockStride + ks * 32) >> 4), idesc, 1u);
+            mma_ss(s_col, qrd + (uint64_t)((ks * 32) >> 4), td + (uint64_t)((2 * L::kBlockStride + ks * 32) >> 4), idesc,
+                   1u);
           mma_commit(smem_u32(&bars->s_full[u % kBrSB]));
           if (u + 1 == ur.u_end) mma_commit(smem_u32(&bars->q_empty));  // the last read of this query
           BR_TRACE(u, kTbQkIssued);
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
   } else if (warp == 2) {
     // ----------------------------------------------------------------- PV
     // PV a unit at a time into O, as soon as every slice of its P is in
-    // TMEM; the commits free the unit's ring entry and its S buffer.
+    // TMEM; the commits free the unit's ring entry and the P buffer.
     SegWalk walk(plan, a.B, maxL);
     int seg = 0;
     uint32_t u_next = 0;
@@ -357,17 +371,15 @@ __global__ void __launch_bounds__(kBrThreads, 1)
           BR_TRACE(u, kTbPSeen);
           const uint32_t k = u % kUnits;
           const uint64_t vd = sdesc_sw128(smem_u32(block_of(0, k, 0)), (uint32_t)L::kBlockStride, 1024);
-          const uint32_t p_base = tmem + kColS + (u % kBrSB) * 128u;
-          // P of tokens 16 ks .. 16 ks + 15 (slice ks / 2): packed columns 32 (ks / 2) + 16 + 8 (ks % 2)
+          // P of tokens 16 ks .. 16 ks + 15: packed columns kColP + 8 ks
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tmem + kColO, p_base + 32u * (ks >> 1) + 16u + 8u * (ks & 1), vd + (uint64_t)((ks * 2048) >> 4),
-                   kIdescPV, (u == ur.u0 && ks == 0) ? 0u : 1u);
+            mma_ts(tmem + kColO, tmem + kColP + 8u * ks, vd + (uint64_t)((ks * 2048) >> 4), kIdescPV,
+                   (u == ur.u0 && ks == 0) ? 0u : 1u);
           if (ur.pages(u) == 2) {
 #pragma unroll
             for (int ks = 4; ks < 8; ++ks)
-              mma_ts(tmem + kColO, p_base + 32u * (ks >> 1) + 16u + 8u * (ks & 1), vd + (uint64_t)((ks * 2048) >> 4),
-                     kIdescPV, 1u);
+              mma_ts(tmem + kColO, tmem + kColP + 8u * ks, vd + (uint64_t)((ks * 2048) >> 4), kIdescPV, 1u);
           }
           mma_commit(smem_u32(&bars->unit_empty[k]));
           mma_commit(smem_u32(&bars->pv_done[u % kBrSB]));
@@ -395,7 +407,8 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     while (ok && walk.next(seq_lens)) {
       if (jq == 0) {
         // the piece's query rows of heads 32q + lane (this branch's 128 latent dims as 64 packed bf16x2
-        // columns, the 64 rope dims as 32) into TMEM, once the previous piece's last QK^T has completed
+        // TMEM columns; the 64 rope dims into the rope query's swizzled row in shared memory), once the
+        // previous piece's last QK^T has completed
         if (seg > 0 && !mbar_wait_warp(smem_u32(&bars->q_empty), (seg - 1) & 1, abort_flag, err, kSiteQEmpty)) break;
         tc_fence_after();
         const __nv_bfloat16* src = q_ws + ((size_t)walk.b * a.H + (real ? head : 0)) * (a.d_c + a.d_r);
@@ -403,8 +416,8 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         const uint4* rop = reinterpret_cast<const uint4*>(src + a.d_c);
         const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int blk = 0; blk < 3; ++blk) {  // latent columns 0-31, 32-63, then the rope's 32
-          const uint4* from = blk < 2 ? lat + 8 * blk : rop;
+        for (int blk = 0; blk < 2; ++blk) {  // latent columns 0-31, 32-63
+          const uint4* from = lat + 8 * blk;
           uint32_t r[32];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -414,8 +427,12 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             r[4 * i + 2] = v.z;
             r[4 * i + 3] = v.w;
           }
-          tmem_st32(tmem + lane_off + (blk < 2 ? kColQ + 32u * blk : kColQR), r);
+          tmem_st32(tmem + lane_off + kColQ + 32u * blk, r);
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)  // 16-byte chunk i of row `head` sits at chunk i ^ (head % 8)
+          *reinterpret_cast<uint4*>(sQR + head * 128 + ((i ^ (head & 7)) * 16)) = real ? __ldg(rop + i) : z;
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
@@ -424,28 +441,50 @@ __global__ void __launch_bounds__(kBrThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       for (uint32_t u = ur.u0; u < ur.u_end; ++u) {
         const int valid = ur.valid(u) - 32 * jq;  // valid tokens of this slice (<= 0: none)
-        // scores of token 32 jq + t at column s_sl + t; its P (bf16) at packed column s_sl + 16 + t / 2
+        // scores of token 32 jq + t at column s_sl + t; its P (bf16) at packed column kColP + 16 jq + t / 2
         const uint32_t s_sl = tmem + lane_off + kColS + (u % kBrSB) * 128u + 32u * (uint32_t)jq;
         if (!mbar_wait_warp(smem_u32(&bars->s_full[u % kBrSB]), (u / kBrSB) & 1, abort_flag, err, kSiteSFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t vhi[16], vlo[16];
-        tmem_ld16(s_sl + 16u, vhi);  // tokens 16-31 of the slice (their columns take the P)
-        tmem_ld16(s_sl, vlo);        // tokens 0-15
+        // the slice's scores (masked past the end of the sequence)
+        float x[32];
+        {
+          uint32_t vhi[16], vlo[16];
+          tmem_ld16(s_sl + 16u, vhi);  // tokens 16-31 of the slice
+          tmem_ld16(s_sl, vlo);        // tokens 0-15
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            x[i] = __uint_as_float(vlo[i]);
+            x[16 + i] = __uint_as_float(vhi[i]);
+          }
+        }
+        if (valid < 32) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i >= valid) x[i] = -INFINITY;
+        }
         float m4[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float x = i < valid ? __uint_as_float(vlo[i]) : -INFINITY;
-          const float y = 16 + i < valid ? __uint_as_float(vhi[i]) : -INFINITY;
-          m4[i & 3] = i < 4 ? fmaxf(x, y) : fmaxf(m4[i & 3], fmaxf(x, y));
-        }
+        for (int i = 0; i < 32; ++i) m4[i & 3] = i < 4 ? x[i] : fmaxf(m4[i & 3], x[i]);
         if (q == 0 && lane == 0) BR_TRACE(u, jq == 0 ? kTbSLoaded : kTbSLoaded1);
         const int rb = (int)(u & 1u);
         bars->red[rb][jq][head] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->red_full[q][rb]));
+        // Past a piece's first unit the running max is known: exponentiate against it (capped at 2^64, so
+        // nothing overflows) while the slices exchange their maxima, and correct afterwards in the rare
+        // case the unit's maximum jumped.  The first unit waits for the exchange.
+        const bool spec = u != ur.u0;
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (spec) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            x[i] = ex2(fminf(x[i] - m_run, kSpecCapLog2));
+            a4[i & 3] += x[i];
+          }
+        }
         if (!mbar_wait_warp(smem_u32(&bars->red_full[q][rb]), (u >> 1) & 1, abort_flag, err, kSiteRed)) {
           ok = false;
           break;
@@ -455,45 +494,60 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         // read the same four values and decide alike
         const float M = fmaxf(fmaxf(bars->red[rb][0][head], bars->red[rb][1][head]),
                               fmaxf(bars->red[rb][2][head], bars->red[rb][3][head]));
-        float m_use, corr;
+        float m_use = m_run, corr = 1.f;
         bool rescale = false;
-        if (u == ur.u0) {
+        if (!spec) {
           m_use = M;
           corr = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            x[i] = ex2(x[i] - M);
+            a4[i & 3] += x[i];
+          }
+        } else if (__any_sync(0xffffffffu, M > m_run + kSpecCapLog2)) {
+          // a jump past the cap (some head of the warp): exponentiate the scores again, read anew from S
+          // (the S buffer is released only below), against each head's new reference
+          rescale = M > m_run + kRescaleLog2;
+          m_use = rescale ? M : m_run;
+          corr = rescale ? ex2(m_run - M) : 1.f;
+          uint32_t vhi[16], vlo[16];
+          tmem_ld16(s_sl + 16u, vhi);
+          tmem_ld16(s_sl, vlo);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float sc = __uint_as_float(i < 16 ? vlo[i] : vhi[i - 16]);
+            x[i] = i < valid ? ex2(sc - m_use) : 0.f;
+            a4[i & 3] = i < 4 ? x[i] : a4[i & 3] + x[i];
+          }
         } else if (M > m_run + kRescaleLog2) {
+          rescale = true;
           m_use = M;
           corr = ex2(m_run - M);
-          rescale = true;
-        } else {
-          m_use = m_run;
-          corr = 1.f;
-        }
-        uint32_t pk[16];
-        float a4[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float p0 = 2 * i < valid ? ex2(__uint_as_float(vlo[2 * i]) - m_use) : 0.f;
-          const float p1 = 2 * i + 1 < valid ? ex2(__uint_as_float(vlo[2 * i + 1]) - m_use) : 0.f;
-          const float p2 = 16 + 2 * i < valid ? ex2(__uint_as_float(vhi[2 * i]) - m_use) : 0.f;
-          const float p3 = 17 + 2 * i < valid ? ex2(__uint_as_float(vhi[2 * i + 1]) - m_use) : 0.f;
-          a4[0] = i == 0 ? p0 : a4[0] + p0;
-          a4[1] = i == 0 ? p1 : a4[1] + p1;
-          a4[2] = i == 0 ? p2 : a4[2] + p2;
-          a4[3] = i == 0 ? p3 : a4[3] + p3;
-          pk[i] = pack_bf16x2(p0, p1);
-          pk[8 + i] = pack_bf16x2(p2, p3);
+          for (int i = 0; i < 32; ++i) x[i] *= corr;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a4[i] *= corr;
         }
-        tmem_st16(s_sl + 16u, pk);  // over the scores of tokens 16-31, read above
+        tc_fence_before();  // the S buffer is read: QK^T of unit u + 2 may overwrite it
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[u % kBrSB]));
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
         l_run = l_run * corr + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
         m_run = m_use;
-        // O is rescaled only when the running max jumped; slice jq takes columns [32 jq, 32 jq + 32)
-        if (__any_sync(0xffffffffu, rescale)) {
-          const uint32_t up = u - 1;  // the previous unit, in this piece since u != u0
+        // the P buffer (and O) are free once PV of the previous unit, of this piece or the last one, is done
+        if (u > 0) {
+          const uint32_t up = u - 1;
           if (!mbar_wait_warp(smem_u32(&bars->pv_done[up % kBrSB]), (up / kBrSB) & 1, abort_flag, err, kSitePvDone)) {
             ok = false;
             break;
           }
           tc_fence_after();
+        }
+        tmem_st16(tmem + lane_off + kColP + 16u * (uint32_t)jq, pk);
+        // O is rescaled only when the running max jumped; slice jq takes columns [32 jq, 32 jq + 32)
+        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             uint32_t o[16];
