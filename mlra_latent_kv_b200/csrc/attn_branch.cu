@@ -242,53 +242,64 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_lat);
       tma_prefetch_desc(&tm_rope);
-      SegWalk walk(plan, a.B, maxL);
-      int* id_ring = bars->page_ids;
-      // ids fetched while the previous unit was issued (pages pend_g, pend_g + 1), parked in the ring at
-      // the next unit, so that a page-table load never sits between a freed ring entry and its refill
-      int pend0 = 0, pend1 = 0, npend = 0;
-      uint32_t pend_g = 0;
-      uint32_t g = 0, u_next = 0;
-      bool ok = true;
-      while (ok && walk.next(seq_lens)) {
-        const UnitRange ur = units_of(walk, u_next);
-        for (uint32_t u = ur.u0; ok && u < ur.u_end; ++u) {
-          const uint32_t k = u % kUnits, use = u / kUnits;
-          if (use > 0 && !mbar_wait(smem_u32(&bars->unit_empty[k]), (use - 1) & 1, abort_flag, err, kSiteStageEmpty)) {
-            ok = false;
-            break;
-          }
-          BR_TRACE(u, kTbStageFree);
-          const int np = ur.pages(u);
-          if (npend > 0) id_ring[pend_g % kIdRing] = pend0;
-          if (npend > 1) id_ring[(pend_g + 1) % kIdRing] = pend1;
-          npend = 0;
-          pend_g = g + kIdAhead;
-          static_assert(kBrUnitPages == 2, "two ids in flight per unit");
-          if (ids.live) {  // the ids of pages g + kIdAhead (+ 1), in flight until the next unit
-            pend0 = ids.fetch(seq_lens, page_table, a.maxp);
-            npend = 1;
-            if (np > 1 && ids.live) {
-              pend1 = ids.fetch(seq_lens, page_table, a.maxp);
-              npend = 2;
-            }
-          }
-          const uint32_t fb = smem_u32(&bars->unit_full[k]);
-          mbar_expect_tx(fb, (uint32_t)(np * 3 * kBrSlot));
-          for (int j = 0; j < np; ++j, ++g) {
-            int pg = id_ring[g % kIdRing];
-            if (pg < 0 || pg >= a.num_pages) {  // reported, and replaced by page 0 so that no load leaves the pool
-              report_error(err, kErrDeviceCheck, walk.b, (ur.first_page(u) + j) * kPage);
-              pg = 0;
-            }
-            tma_load_2d(smem_u32(block_of(0, k, j)), &tm_lat, fb, d_cb * br, pg * kPage);
-            tma_load_2d(smem_u32(block_of(1, k, j)), &tm_lat, fb, d_cb * br + 64, pg * kPage);
-            tma_load_2d(smem_u32(block_of(2, k, j)), &tm_rope, fb, 0, pg * kPage);
-          }
-          BR_TRACE(u, kTbTma);
+    }
+    // The whole warp walks the pages (every lane keeps the same cursors); per
+    // unit, lane j fetches the id of page g + kIdAhead + j and parks it in the
+    // ring at the next unit, and lane 3 j + s issues block s of the unit's
+    // page j, so that a unit costs the warp a few instructions, not a few
+    // dozen dependent ones on one lane.
+    SegWalk walk(plan, a.B, maxL);
+    int* id_ring = bars->page_ids;
+    int pend = 0;          // this lane's fetched id (of page pend_g + lane), parked at the next unit
+    int npend = 0;
+    uint32_t pend_g = 0;
+    uint32_t g = 0, u_next = 0;
+    bool ok = true;
+    while (ok && walk.next(seq_lens)) {
+      const UnitRange ur = units_of(walk, u_next);
+      for (uint32_t u = ur.u0; u < ur.u_end; ++u) {
+        const uint32_t k = u % kUnits, use = u / kUnits;
+        if (use > 0 && !mbar_wait_warp(smem_u32(&bars->unit_empty[k]), (use - 1) & 1, abort_flag, err, kSiteStageEmpty)) {
+          ok = false;
+          break;
         }
-        u_next = ur.u_end;
+        if (lane == 0) BR_TRACE(u, kTbStageFree);
+        const int np = ur.pages(u);
+        if (lane < npend) id_ring[(pend_g + lane) % kIdRing] = pend;
+        {
+          int my_b = -1, my_p = 0, nf = 0;
+#pragma unroll
+          for (int j = 0; j < kBrUnitPages; ++j)
+            if (j < np && ids.live) {
+              if (lane == j) {
+                my_b = ids.w.b;
+                my_p = ids.p;
+              }
+              ids.step(seq_lens);
+              ++nf;
+            }
+          if (lane < nf) pend = __ldg(page_table + (size_t)my_b * a.maxp + my_p);
+          npend = nf;
+          pend_g = g + kIdAhead;
+        }
+        const uint32_t fb = smem_u32(&bars->unit_full[k]);
+        if (lane == 0) mbar_expect_tx(fb, (uint32_t)(np * 3 * kBrSlot));
+        __syncwarp();
+        if (lane < 3 * np) {
+          const int j = lane / 3, s2 = lane % 3;
+          int pg = id_ring[(g + (uint32_t)j) % kIdRing];
+          if (pg < 0 || pg >= a.num_pages) {  // reported, and replaced by page 0 so that no load leaves the pool
+            report_error(err, kErrDeviceCheck, walk.b, (ur.first_page(u) + j) * kPage);
+            pg = 0;
+          }
+          tma_load_2d(smem_u32(block_of(s2, k, j)), s2 < 2 ? &tm_lat : &tm_rope, fb, s2 < 2 ? d_cb * br + 64 * s2 : 0,
+                      pg * kPage);
+        }
+        __syncwarp();
+        if (lane == 0) BR_TRACE(u, kTbTma);
+        g += (uint32_t)np;
       }
+      u_next = ur.u_end;
     }
   } else if (warp == 1) {
     // --------------------------------------------------------------- QK^T
