@@ -328,3 +328,34 @@ def test_workload_kernel_family(name):
     s.step()
     torch.cuda.synchronize()
     s.check()
+
+
+@pytest.mark.parametrize("G", [1, 2])
+@pytest.mark.parametrize("logit", [30.0, 120.0])
+def test_mlra4_max_jump_after_the_first_unit(logit, G):
+    """MLRA-4 on the branch kernel, whose softmax exponentiates against the
+    running max before a unit's maximum is known: a key planted well past the
+    first two pages, ``logit`` natural-log units above head 0's others in every
+    branch (30: a jump the kernel corrects by scaling; 120 = 173 log2 units:
+    past its 2^64 cap, so it exponentiates that unit again).  Other heads see
+    the key at random, smaller offsets, so heads with and without a jump share
+    a warp."""
+    w = synth.workload("mlra4").with_(B=1, H=128, seq_len=1000, seq_len_range=None)
+    inp = synth.make_inputs(w)
+    inp["q_rope"].zero_()
+    scale = 1.0 / np.sqrt(w.d_h + w.d_r)
+    t = int(np.where(inp["tok_pos"].numpy() == 700)[0][0])
+    d_cb = w.d_c // w.n_branch
+    c = inp["c_kv"][t].double().clone()
+    for br in range(w.n_branch):
+        q_lat = inp["q_nope"][0, 0].double() @ inp["W_UK"][0][:, br * d_cb:(br + 1) * d_cb].double()
+        c[br * d_cb:(br + 1) * d_cb] = q_lat / (q_lat @ q_lat) * (logit / scale)
+    inp["c_kv"][t] = c.to(inp["c_kv"].dtype)
+    s = DecodeSession(w, inp, num_splits=G)
+    assert "branch" in s.plan()["attention"], s.plan()
+    out = s.step().clone()
+    torch.cuda.synchronize()
+    s.check()
+    ref = oracle.decode(oracle_inputs(w, inp))
+    err, tol = compare(out, ref)
+    assert err <= tol, f"logit={logit} G={G}: {err:.3e} > {tol:.3e} (rel l2 {rel_l2(out, ref):.2e})"
