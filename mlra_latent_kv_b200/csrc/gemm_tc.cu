@@ -181,17 +181,18 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------------------------------
 // a4 + a5: split combine fused into the output up-projection.
-// grid (H, d_v / 128, ceil(B / kCuRows)), block 512: a CTA takes one head, 128
-// value dims and a block of kCuRows sequences, so that a few heads still fill
+// grid (H, d_v / 128, ceil(B / R)), block 512: a CTA takes one head, 128 value
+// dims and a block of R sequences (16, or 32 when the heads alone nearly fill
+// the GPU: more CTAs would re-read the weights for no gain), so that a few heads still fill
 // the GPU (at H = 32 one CTA per head would leave most SMs idle, each of its
 // CTAs streaming a whole head's partials).
 //   A (M = 128 value dims, K = d_c)      = W_UV[h][:, m0:m0+128]  MN-major (TMA)
-//   B (N = kCuRows batch rows, K = d_c)  = o_lat[b0 + n, h, :] built here in smem:
+//   B (N = R batch rows, K = d_c)        = o_lat[b0 + n, h, :] built here in smem:
 //       o_lat[b, h, br cols] = branch_scale * sum_s 2^(m_s - M) o_s / L
-//   D (TMEM, 128 lanes x kCuRows)        -> out[b][h][m0 + lane] (bf16)
+//   D (TMEM, 128 lanes x R)              -> out[b][h][m0 + lane] (bf16)
 // ---------------------------------------------------------------------------
 constexpr int kCuThreads = 512;
-constexpr int kCuRows = 16;      // sequences per CTA (the MMA's N)
+constexpr int kCuRowsMax = 32;   // sequences per CTA at most (the MMA's N)
 constexpr int kPieceUnroll = 4;  // partials of a row fetched together
 
 __global__ void __launch_bounds__(kCuThreads, 1)
@@ -202,9 +203,9 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int a_bytes = 2 * a.K * 128;             // K = d_c rows, two 64-column M blocks
   const int n_ml = (a.G + a.B - 1) * a.n_branch;  // (slot, branch) pairs
-  uint8_t* sB = smem + a_bytes;                  // d_c/64 blocks of kCuRows rows
+  uint8_t* sB = smem + a_bytes;                  // d_c/64 blocks of R rows
   uint8_t* sA = smem;
-  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * kCuRows * 128);  // [slot][n_branch] piece weights
+  float* s_wt = reinterpret_cast<float*>(sB + (a.K / 64) * a.R * 128);  // [slot][n_branch] piece weights
   float* s_m = s_wt + n_ml;                                              // [slot][n_branch] running max
   float* s_l = s_m + n_ml;                                               // [slot][n_branch] sum
   int* s_c0 = reinterpret_cast<int*>(s_l + n_ml);
@@ -214,10 +215,10 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   __shared__ long long s_T;
-  const int h = blockIdx.x, m0 = blockIdx.y * 128, b0 = blockIdx.z * kCuRows;
-  const int nb = min(kCuRows, a.B - b0);  // sequences of this CTA
+  const int h = blockIdx.x, m0 = blockIdx.y * 128, b0 = blockIdx.z * a.R;
+  const int nb = min(a.R, a.B - b0);  // sequences of this CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = tmem_cols_for(kCuRows);
+  const uint32_t ncols = tmem_cols_for(a.R);
   const int maxL = a.maxp * kPage;
   GEMM_TRACE(1, 0);
   if (threadIdx.x == 0) {
@@ -310,14 +311,14 @@ __global__ void __launch_bounds__(kCuThreads, 1)
   // the partials of up to kPieceUnroll pieces of both before using any.
   const int chunks = a.K / 8;
   const int d_cb = a.K / a.n_branch;
-  const int n_items = kCuRows * chunks;
+  const int n_items = a.R * chunks;
   for (int base = threadIdx.x; base < n_items; base += 2 * blockDim.x) {
     int rq[2], bq[2], chq[2], c0q[2], c1q[2], brq[2];  // local row, sequence, chunk, workers, branch
     float acc[2][8];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int idx = base + u * blockDim.x;
-      rq[u] = idx < n_items ? idx / chunks : kCuRows;
+      rq[u] = idx < n_items ? idx / chunks : a.R;
       bq[u] = b0 + rq[u];
       chq[u] = idx % chunks;
       const bool row = rq[u] < nb;
@@ -363,13 +364,13 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      if (rq[u] >= kCuRows) continue;
+      if (rq[u] >= a.R) continue;
       uint4 pk;  // rows past the batch are zero (no pieces, weights 0)
       pk.x = pack_bf16x2(acc[u][0], acc[u][1]);
       pk.y = pack_bf16x2(acc[u][2], acc[u][3]);
       pk.z = pack_bf16x2(acc[u][4], acc[u][5]);
       pk.w = pack_bf16x2(acc[u][6], acc[u][7]);
-      *reinterpret_cast<uint4*>(sB + (chq[u] / 8) * kCuRows * 128 + sw128_off(rq[u], chq[u] % 8)) = pk;
+      *reinterpret_cast<uint4*>(sB + (chq[u] / 8) * a.R * 128 + sw128_off(rq[u], chq[u] % 8)) = pk;
     }
   }
   fence_proxy_async_smem();
@@ -379,10 +380,10 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     if (mbar_wait(smem_u32(&full_bar), 0, &abort_flag, err, 22)) {
       GEMM_TRACE(1, 4);
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, kCuRows, true, false);
+      const uint32_t idesc = idesc_bf16_f32(128, a.R, true, false);
       const uint64_t ad0 = sdesc_sw128(smem_u32(sA), a.K * 128, 1024);
       const uint64_t bd0 = sdesc_sw128(smem_u32(sB), 16, 1024);
-      const uint64_t bkb = (uint64_t)((kCuRows * 128) >> 4);
+      const uint64_t bkb = (uint64_t)((a.R * 128) >> 4);
       for (int kb = 0; kb < a.K / 64; ++kb) {
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
@@ -396,13 +397,15 @@ __global__ void __launch_bounds__(kCuThreads, 1)
     GEMM_TRACE(1, 5);
     tc_fence_after();
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    static_assert(kCuRows == 16, "one 16-column TMEM load per lane quarter");
-    uint32_t v[16];
-    tmem_ld16(tmem + lane_off, v);
+    for (int cc = 0; cc < a.R; cc += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_off + (uint32_t)cc, v);
 #pragma unroll
-    for (int j = 0; j < kCuRows; ++j)
-      if (j < nb)
-        out[((size_t)(b0 + j) * a.H + h) * a.N_out + m0 + warp * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[j]));
+      for (int j = 0; j < 16; ++j)
+        if (cc + j < nb)
+          out[((size_t)(b0 + cc + j) * a.H + h) * a.N_out + m0 + warp * 32 + lane] =
+              __float2bfloat16_rn(__uint_as_float(v[j]));
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -422,11 +425,17 @@ bool absorb_tc_supported(int dtype, int B, int d_h, int d_c) {
 
 int batch_pad(int B) { return B <= 16 ? 16 : (B + 15) / 16 * 16; }
 
-// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B), d_c/64 x kCuRows x
-// 128 B of o_lat rows, the (m, l, weight) of every slot and branch, two ints
-// per sequence, one flag per worker
+// Sequences per CTA: 16, or up to 32 when the heads and value blocks alone
+// give most of a wave of CTAs (then a finer split only re-reads the weights).
+static int combine_rows(int B, int H, int d_v) {
+  return H * (d_v / 128) >= 96 ? (batch_pad(B) < kCuRowsMax ? batch_pad(B) : kCuRowsMax) : 16;
+}
+
+// shared memory: the whole W_UV[h] slice (2 x d_c x 128 B), d_c/64 x R x 128 B
+// of o_lat rows (R at most kCuRowsMax), the (m, l, weight) of every slot and
+// branch, two ints per sequence, one flag per worker
 static size_t upproj_smem_bytes(int B, int d_c, int G, int n_branch) {
-  return 1024 + (size_t)2 * d_c * 128 + (size_t)(d_c / 64) * kCuRows * 128 +
+  return 1024 + (size_t)2 * d_c * 128 + (size_t)(d_c / 64) * kCuRowsMax * 128 +
          (size_t)3 * (G + B) * n_branch * 4 + (size_t)2 * B * 4 + (size_t)G * 4;
 }
 
@@ -455,11 +464,13 @@ cudaError_t launch_combine_upproj_tc(const float* o_part, const float* ml_part, 
   CUtensorMap tw;
   if (!tmap_2d(&tw, W_UV, (uint64_t)a.N_out, (uint64_t)a.H * a.K, 64, (uint32_t)(a.K < 256 ? a.K : 256)))
     return cudaErrorInvalidValue;
+  GemmArgs g = a;
+  g.R = combine_rows(a.B, a.H, a.N_out);
   const int smem = (int)upproj_smem_bytes(a.B, a.K, a.G, a.n_branch);
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(combine_upproj_tc_kernel), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.H, a.N_out / 128, (a.B + kCuRows - 1) / kCuRows);
+  cfg.gridDim = dim3(g.H, g.N_out / 128, (g.B + g.R - 1) / g.R);
   cfg.blockDim = dim3(kCuThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -469,7 +480,7 @@ cudaError_t launch_combine_upproj_tc(const float* o_part, const float* ml_part, 
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, combine_upproj_tc_kernel, tw, o_part, ml_part, seq_lens, (__nv_bfloat16*)out, err,
-                            a);
+                            g);
 }
 
 #ifdef MLRA_TRACE

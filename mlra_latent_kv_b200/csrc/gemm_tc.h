@@ -17,6 +17,7 @@ struct GemmArgs {
   int G, n_branch, maxp;
   float branch_scale;
   float q_scale;   // absorption only: multiplies q_lat and the rotated q_rope before rounding
+  int R;           // combine + up-projection only: sequences per CTA (the MMA's N; 16 or 32)
 };
 
 int batch_pad(int B);
