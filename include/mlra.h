@@ -170,6 +170,41 @@ MLRA_API mlra_status mlra_decode_host(const mlra_dims* dims, const void* h_q_nop
                                       const int32_t* page_table, const int32_t* h_seq_lens, void* h_out,
                                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* FP8 latent cache (an extension: yunthe.com, "多头潜在注意力机制：内存优化与推理
+ * 加速的革新方案", section "一、技术演进背景", names 8-bit quantization of the
+ * KV cache as a way to shrink it, at some cost in precision; the format below
+ * is this library's reading, as the page fixes none).
+ *
+ * Format: every element of latent_cache [P,64,d_c] and rope_cache [P,64,d_r]
+ * is one FP8 E4M3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities, S.1111.111 = NaN, largest finite 448) in a uint8_t, and each
+ * page of each tensor has one fp32 scale: value = decode(code) * scale[page].
+ *
+ * mlra_quantize_pages_fp8 -- quantize a bf16 (dims->dtype = MLRA_BF16) or
+ * fp32 pool of dims->num_pages pages: scale = (largest finite |x| on the page)
+ * / 448 in fp32 (1 for a page with no nonzero finite value); code = E4M3 of
+ * fl32(x / scale), nearest with ties to even, saturating at +-448; NaN stays
+ * NaN.  Outputs: latent_fp8 [P,64,d_c] and rope_fp8 [P,64,d_r] bytes,
+ * latent_scale [P] and rope_scale [P] fp32 (4-byte aligned), all device
+ * memory owned by the caller.  Asynchronous on `stream`; returns
+ * MLRA_ERR_INVALID_ARG for a NULL pointer.
+ *
+ * mlra_decode_fp8 -- mlra_decode over such a cache: the same arguments, with
+ * the FP8 pools and their scales in place of latent_cache and rope_cache.  It
+ * runs on the CUDA-core kernels (fp32 arithmetic on the dequantized values);
+ * dims->kernel = MLRA_KERNEL_TC is refused with MLRA_ERR_UNSUPPORTED.
+ *   workspace: >= mlra_workspace_bytes() of the same dims with kernel =
+ *   MLRA_KERNEL_SIMT, 256-byte aligned. */
+MLRA_API mlra_status mlra_quantize_pages_fp8(const mlra_dims* dims, const void* latent_cache,
+                                             const void* rope_cache, uint8_t* latent_fp8, uint8_t* rope_fp8,
+                                             float* latent_scale, float* rope_scale, cudaStream_t stream);
+MLRA_API mlra_status mlra_decode_fp8(const mlra_dims* dims, const void* q_nope, const void* q_rope,
+                                     const int32_t* q_pos, const void* W_UK, const void* W_UV,
+                                     const uint8_t* latent_fp8, const uint8_t* rope_fp8,
+                                     const float* latent_scale, const float* rope_scale,
+                                     const int32_t* page_table, const int32_t* seq_lens, void* out,
+                                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* mlra_describe_plan -- the kernels mla_decode / mlra_decode launch for
  * `dims`, as one NUL-terminated line of ';'-separated key=value fields:
  *   family     tcgen05 | tcgen05+cuda-core | cuda-core (kernel AUTO picks

@@ -64,6 +64,8 @@ SIGNATURES = {
     "mlra_attend_partial": (ctypes.c_int, [_DIMS, _P, _P, _I32P, _P, _P, _P, _I32P, _I32P, _P, _P, _P, _SZ, _P]),
     "mlra_merge_workspace_bytes": (_SZ, [_DIMS]),
     "mlra_merge_upproj": (ctypes.c_int, [_DIMS, ctypes.c_int, _P, _P, _P, _P, _P, _SZ, _P]),
+    "mlra_quantize_pages_fp8": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P]),
+    "mlra_decode_fp8": (ctypes.c_int, [_DIMS, _P, _P, _I32P, _P, _P, _P, _P, _P, _P, _I32P, _I32P, _P, _P, _SZ, _P]),
     "mlra_check_status": (ctypes.c_int, [_P, _P]),
     "mlra_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_longlong, _P]),
     "mlra_last_error": (ctypes.c_char_p, []),
@@ -144,6 +146,23 @@ def merge_upproj(dims, o_parts, lse_parts, W_UV, out, workspace, stream=None):
     _check(lib().mlra_merge_upproj(ctypes.byref(dims), int(o_parts.shape[0]), _ptr(o_parts), _ptr(lse_parts),
                                    _ptr(W_UV), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def quantize_pages_fp8(dims, latent_cache, rope_cache, latent_fp8, rope_fp8, latent_scale, rope_scale,
+                       stream=None):
+    """FP8 E4M3 codes and per-page fp32 scales of a bf16/fp32 pool (see include/mlra.h)."""
+    _check(lib().mlra_quantize_pages_fp8(ctypes.byref(dims), _ptr(latent_cache), _ptr(rope_cache), _ptr(latent_fp8),
+                                         _ptr(rope_fp8), _ptr(latent_scale), _ptr(rope_scale), _stream(stream)))
+
+
+def decode_fp8(dims, q_nope, q_rope, q_pos, W_UK, W_UV, latent_fp8, rope_fp8, latent_scale, rope_scale, page_table,
+               seq_lens, out, workspace, stream=None):
+    """mlra_decode over an FP8 cache (CUDA-core kernels; the workspace is sized for kernel SIMT)."""
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().mlra_decode_fp8(ctypes.byref(dims), _ptr(q_nope), _ptr(q_rope), _ptr(q_pos), _ptr(W_UK), _ptr(W_UV),
+                                 _ptr(latent_fp8), _ptr(rope_fp8), _ptr(latent_scale), _ptr(rope_scale),
+                                 _ptr(page_table), _ptr(seq_lens), _ptr(out), _ptr(workspace), nbytes,
+                                 _stream(stream)))
 
 
 def workspace_bytes(dims: Dims) -> int:

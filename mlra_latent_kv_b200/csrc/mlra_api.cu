@@ -141,12 +141,28 @@ struct PartialOut {
   float* lse;
 };
 
+// An FP8 cache: E4M3 codes in latent_cache/rope_cache, one fp32 scale per page
+// of each.  Its decode runs on the CUDA-core kernels.
+struct Fp8Scales {
+  const float* lat;
+  const float* rop;
+};
+
 mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, const void* q_rope,
                         const int32_t* q_pos, const void* W_UK, const void* W_UV, const void* latent_cache,
                         const void* rope_cache, const int32_t* page_table, const int32_t* seq_lens, void* out,
                         void* workspace, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* ev,
-                        const PartialOut* part = nullptr) {
+                        const PartialOut* part = nullptr, const Fp8Scales* fp8 = nullptr) {
   DecodePlan p;
+  mlra_dims dsimt;
+  if (fp8) {  // the FP8 cache is read by the CUDA-core attention kernel
+    if (!fp8->lat || !fp8->rop) return fail(MLRA_ERR_INVALID_ARG, "FP8 scales are NULL");
+    if (!aligned(fp8->lat, 4) || !aligned(fp8->rop, 4)) return fail(MLRA_ERR_INVALID_ARG, "FP8 scales not 4-byte aligned");
+    if (d->kernel == MLRA_KERNEL_TC) return fail(MLRA_ERR_UNSUPPORTED, "the FP8 cache runs on the CUDA-core kernels");
+    dsimt = *d;
+    dsimt.kernel = MLRA_KERNEL_SIMT;
+    d = &dsimt;
+  }
   mlra_status st = make_plan(d, &p);
   if (st != MLRA_OK) return st;
   if (mla_only && d->n_branch != 1) return fail(MLRA_ERR_INVALID_ARG, "mla_decode needs n_branch=1 (use mlra_decode)");
@@ -204,6 +220,11 @@ mlra_status decode_impl(const mlra_dims* d, bool mla_only, const void* q_nope, c
     e = launch_attend_tc(q_ws, latent_cache, rope_cache, page_table, seq_lens, o_part, ml_part, err, at, stream,
                          tc_absorb && ev == nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 attention launch");
+  } else if (fp8) {
+    e = launch_attend_simt_fp8(static_cast<const float*>(q_ws), static_cast<const uint8_t*>(latent_cache),
+                               static_cast<const uint8_t*>(rope_cache), fp8->lat, fp8->rop, page_table, seq_lens,
+                               o_part, ml_part, err, at, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "FP8 attention launch");
   } else {
     e = launch_attend_simt(d->dtype, static_cast<const float*>(q_ws), latent_cache, rope_cache, page_table, seq_lens,
                            o_part, ml_part, err, at, stream);
@@ -280,6 +301,35 @@ mlra_status mlra_decode(const mlra_dims* dims, const void* q_nope, const void* q
                         size_t workspace_bytes, cudaStream_t stream) {
   return decode_impl(dims, false, q_nope, q_rope, q_pos, W_UK, W_UV, latent_cache, rope_cache, page_table, seq_lens,
                      out, workspace, workspace_bytes, stream, nullptr);
+}
+
+mlra_status mlra_quantize_pages_fp8(const mlra_dims* dims, const void* latent_cache, const void* rope_cache,
+                                    uint8_t* latent_fp8, uint8_t* rope_fp8, float* latent_scale, float* rope_scale,
+                                    cudaStream_t stream) {
+  mlra_status st = check_dims(dims);
+  if (st != MLRA_OK) return st;
+  const void* ptrs[] = {latent_cache, rope_cache, latent_fp8, rope_fp8, latent_scale, rope_scale};
+  const char* names[] = {"latent_cache", "rope_cache", "latent_fp8", "rope_fp8", "latent_scale", "rope_scale"};
+  for (int i = 0; i < 6; ++i)
+    if (!ptrs[i]) return fail(MLRA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+  if (!aligned(latent_scale, 4) || !aligned(rope_scale, 4)) return fail(MLRA_ERR_INVALID_ARG, "scales not 4-byte aligned");
+  cudaError_t e = launch_quantize_pages(dims->dtype, latent_cache, dims->num_pages, kPage * dims->d_c, latent_fp8,
+                                        latent_scale, stream);
+  if (e == cudaSuccess)
+    e = launch_quantize_pages(dims->dtype, rope_cache, dims->num_pages, kPage * dims->d_r, rope_fp8, rope_scale,
+                              stream);
+  if (e != cudaSuccess) return cuda_fail(e, "FP8 quantizer launch");
+  return MLRA_OK;
+}
+
+mlra_status mlra_decode_fp8(const mlra_dims* dims, const void* q_nope, const void* q_rope, const int32_t* q_pos,
+                            const void* W_UK, const void* W_UV, const uint8_t* latent_fp8, const uint8_t* rope_fp8,
+                            const float* latent_scale, const float* rope_scale, const int32_t* page_table,
+                            const int32_t* seq_lens, void* out, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  const Fp8Scales sc{latent_scale, rope_scale};
+  return decode_impl(dims, false, q_nope, q_rope, q_pos, W_UK, W_UV, latent_fp8, rope_fp8, page_table, seq_lens, out,
+                     workspace, workspace_bytes, stream, nullptr, nullptr, &sc);
 }
 
 mlra_status mlra_decode_profiled(const mlra_dims* dims, const void* q_nope, const void* q_rope, const int32_t* q_pos,

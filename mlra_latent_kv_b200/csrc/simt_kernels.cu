@@ -2,6 +2,8 @@
 // attention, split combine and output up-projection.  They run every shape
 // the ABI accepts (fp32 and bf16) and are the path for shapes the tcgen05
 // kernels do not implement.  Arithmetic is fp32 throughout.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -84,6 +86,16 @@ __global__ void __launch_bounds__(128) absorb_kernel(const T* __restrict__ q_nop
 // head reads each piece's row contiguously), ml_part[slot][n_branch][2][H] (m, l).
 // ---------------------------------------------------------------------------
 constexpr int kTileTok = 16;
+
+// Cache element -> fp32.  An FP8 cache (E4M3 codes, one fp32 scale per page
+// and tensor) stores uint8_t; its value is decode(code) * scale[page].
+__device__ __forceinline__ float cache_f(float x, const float*, int) { return x; }
+__device__ __forceinline__ float cache_f(__nv_bfloat16 x, const float*, int) { return __bfloat162float(x); }
+__device__ __forceinline__ float cache_f(uint8_t x, const float* scale, int pg) {
+  __nv_fp8_e4m3 v;
+  v.__x = x;
+  return static_cast<float>(v) * __ldg(scale + pg);
+}
 constexpr int kMaxDpl = 16;  // d_c <= 512
 constexpr int kMaxRpl = 2;   // d_r <= 64
 constexpr int kMaxBr = 8;
@@ -93,7 +105,8 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(const float* __restric
                                                           const T* __restrict__ rop, const int* __restrict__ page_table,
                                                           const int* __restrict__ seq_lens, float* __restrict__ o_part,
                                                           float* __restrict__ ml_part, int* __restrict__ err,
-                                                          AttnArgs a) {
+                                                          AttnArgs a, const float* __restrict__ lat_scale = nullptr,
+                                                          const float* __restrict__ rop_scale = nullptr) {
   extern __shared__ float tile[];  // [kTileTok][d_c + d_r]
   __shared__ WorkerPlan s_plan;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,7 +156,8 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(const float* __restric
         const int t = tt + j;
         const int pg = page_of(page_table, a.maxp, a.num_pages, b, t, err);
         const size_t slot = (size_t)pg * kPage + (t % kPage);
-        tile[j * W + col] = col < a.d_c ? to_f(lat[slot * a.d_c + col]) : to_f(rop[slot * a.d_r + (col - a.d_c)]);
+        tile[j * W + col] = col < a.d_c ? cache_f(lat[slot * a.d_c + col], lat_scale, pg)
+                                        : cache_f(rop[slot * a.d_r + (col - a.d_c)], rop_scale, pg);
       }
       __syncthreads();
       if (h < a.H) {
@@ -332,6 +346,60 @@ cudaError_t launch_attend_simt(int dtype, const float* q_ws, const void* lat, co
     attend_simt_kernel<float><<<grid, 256, smem, st>>>(q_ws, (const float*)lat, (const float*)rop, page_table,
                                                       seq_lens, o_part, ml_part, err, a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attend_simt_fp8(const float* q_ws, const uint8_t* lat, const uint8_t* rop, const float* lat_scale,
+                                   const float* rop_scale, const int* page_table, const int* seq_lens, float* o_part,
+                                   float* ml_part, int* err, const AttnArgs& a, cudaStream_t st) {
+  dim3 grid(a.G, (a.H + 7) / 8);
+  size_t smem = (size_t)kTileTok * (a.d_c + a.d_r) * sizeof(float);
+  attend_simt_kernel<uint8_t><<<grid, 256, smem, st>>>(q_ws, lat, rop, page_table, seq_lens, o_part, ml_part, err, a,
+                                                       lat_scale, rop_scale);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// FP8 cache quantizer: one CTA per page of one tensor (latent or rope).
+//   scale = (largest finite |x| on the page) / 448, fp32 (1 for a page with no
+//   nonzero finite value); code = E4M3 of fl32(x / scale), nearest with ties
+//   to even, saturating at 448; NaN stays NaN.
+// grid (num_pages), block 256.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_pages_kernel(const T* __restrict__ pool, int n_per_page,
+                                                             uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  __shared__ float red[8];
+  __shared__ float s_scale;
+  const T* src = pool + (size_t)blockIdx.x * n_per_page;
+  uint8_t* dst = codes + (size_t)blockIdx.x * n_per_page;
+  float amax = 0.f;
+  for (int i = threadIdx.x; i < n_per_page; i += blockDim.x) {
+    const float v = to_f(src[i]);
+    if (isfinite(v)) amax = fmaxf(amax, fabsf(v));
+  }
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    s_scale = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+    scales[blockIdx.x] = s_scale;
+  }
+  __syncthreads();
+  const float scale = s_scale;
+  for (int i = threadIdx.x; i < n_per_page; i += blockDim.x)
+    dst[i] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(to_f(src[i]), scale), __NV_SATFINITE, __NV_E4M3);
+}
+
+cudaError_t launch_quantize_pages(int dtype, const void* pool, int num_pages, int n_per_page, uint8_t* codes,
+                                  float* scales, cudaStream_t st) {
+  if (dtype == 1)
+    quantize_pages_kernel<__nv_bfloat16><<<num_pages, 256, 0, st>>>((const __nv_bfloat16*)pool, n_per_page, codes,
+                                                                    scales);
+  else
+    quantize_pages_kernel<float><<<num_pages, 256, 0, st>>>((const float*)pool, n_per_page, codes, scales);
   return cudaGetLastError();
 }
 

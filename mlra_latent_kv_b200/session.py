@@ -93,6 +93,29 @@ class DecodeSession:
                             self.latent_cache, self.rope_cache, self.page_table, self.seq_lens, self.out,
                             self.workspace, stream=stream)
 
+    def quantize_fp8(self, stream=None):
+        """Quantize the cache pools to FP8 E4M3 with per-page scales (mlra_quantize_pages_fp8) and size
+        the CUDA-core workspace that mlra_decode_fp8 needs."""
+        dev = self.device
+        self.lat8 = torch.empty(self.latent_cache.shape, dtype=torch.uint8, device=dev)
+        self.rop8 = torch.empty(self.rope_cache.shape, dtype=torch.uint8, device=dev)
+        self.lat_scale = torch.empty(self.num_pages, dtype=torch.float32, device=dev)
+        self.rop_scale = torch.empty(self.num_pages, dtype=torch.float32, device=dev)
+        abi.quantize_pages_fp8(self.dims, self.latent_cache, self.rope_cache, self.lat8, self.rop8, self.lat_scale,
+                               self.rop_scale, stream=stream)
+        d = self.dims
+        self.dims_fp8 = abi.make_dims(B=d.B, H=d.H, d_h=d.d_h, d_v=d.d_v, d_c=d.d_c, d_r=d.d_r,
+                                      max_pages_per_seq=d.max_pages_per_seq, num_pages=d.num_pages,
+                                      n_branch=d.n_branch, branch_scale=d.branch_scale, rope_base=d.rope_base,
+                                      dtype=self.w.dtype, num_splits=d.num_splits, kernel="simt")
+        self.ws_fp8 = torch.zeros(abi.workspace_bytes(self.dims_fp8), dtype=torch.uint8, device=dev)
+
+    def decode_fp8(self, stream=None):
+        """One decode over the FP8 pools made by quantize_fp8 (into self.out)."""
+        abi.decode_fp8(self.dims_fp8, self.q_nope, self.q_rope, self.q_pos, self.W_UK, self.W_UV, self.lat8, self.rop8,
+                       self.lat_scale, self.rop_scale, self.page_table, self.seq_lens, self.out, self.ws_fp8,
+                       stream=stream)
+
     def decode_host(self, h_q_nope, h_q_rope, h_q_pos, h_seq_lens, h_out, stream=None):
         """One decode through the host-buffer entry point (inputs in, output out, on `stream`)."""
         if getattr(self, "host_ws", None) is None:

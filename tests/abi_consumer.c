@@ -28,6 +28,7 @@ static void* const entry_points[] = {
     (void*)mlra_selftest_wait_timeout, (void*)mlra_check_status, (void*)mlra_last_error,
     (void*)mlra_shutdown,         (void*)mlra_version,          (void*)mlra_describe_plan,
     (void*)mlra_attend_partial,   (void*)mlra_merge_workspace_bytes, (void*)mlra_merge_upproj,
+    (void*)mlra_quantize_pages_fp8, (void*)mlra_decode_fp8,
 };
 
 static mlra_dims dims_dsv2(void) {
