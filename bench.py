@@ -506,6 +506,72 @@ def run_ours(args, w):
     return 0
 
 
+def run_fp8(args, w):
+    """The step over an FP8 E4M3 cache (one fp32 scale per page and tensor), quantized from the workload's
+    bf16 cache by mlra_quantize_pages_fp8 and decoded by mlra_decode_fp8 on the CUDA-core kernels.
+    Timed as whole steps (no stage events in that entry point); the roofline is the one of the FP8 cache
+    bytes, half of the bf16 ones, against the whole step's time."""
+    from mlra_latent_kv_b200 import abi
+    from mlra_latent_kv_b200.session import DecodeSession
+    rank, ws, local = mdist.world()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    mdist.init("nccl" if ws > 1 else "gloo")
+    wr = w.with_(seed=mdist.rank_seed(w.seed, rank))
+    if wr.append_d_model:
+        raise SystemExit("--cache fp8 takes a workload without append")
+    inp = synth.make_inputs(wr)
+    sess = DecodeSession(wr, inp, device=dev)
+    sess.quantize_fp8()
+    sb = step_bytes(wr, inp)
+    cache8 = sb["tokens"] * (wr.d_c + wr.d_r) + 2 * 4 * int(inp["num_pages"])  # codes + per-page scales
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        flush.fill_(1)
+        sess.decode_fp8()
+    torch.cuda.synchronize(dev)
+    abi.check_status(sess.ws_fp8)
+    starts, ends = _events(K), _events(K)
+    mdist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            sess.decode_fp8()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / K
+    ms = mdist.max_over_ranks(ms, dev)
+    peaks, src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    gbs = cache8 / (ms * 1e-3) / 1e9
+    plan = abi.describe_plan(sess.dims_fp8)
+    line = {
+        "metric": "latent decode over an FP8 latent cache: µs/step, achieved HBM GB/s of the FP8 cache bytes",
+        "value": (cache8 + sb["weights"]) * ws / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": ws, "steps": K,
+        "warmup": W, "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8 e4m3 cache, fp32 compute",
+        "data": "synthetic (seeded per workload), the bf16 cache quantized per page",
+        "config": {"workload": wr.name, "cache": "fp8_e4m3, one fp32 scale per page and tensor", "B": wr.B,
+                   "H": wr.H, "d_c": wr.d_c, "d_r": wr.d_r, "n_branch": wr.n_branch,
+                   "tokens_attended": sb["tokens"], "l2": "flushed: 256 MiB written before every timed step"},
+        "roofline": {"kernel": "whole decode step over the FP8 cache (CUDA-core kernels)", "bound": "hbm",
+                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_source": ("of measured" if src == "measured" else "of fallback") + " (hbm_gbs)",
+                     "algorithmic_bytes_per_launch": cache8, "bf16_cache_bytes": sb["cache"],
+                     "roofline_us": cache8 / (hbm * 1e9) * 1e6, "traffic": None},
+        "gpu_launches": K * int(plan.get("kernels", 4)), "kernels": plan, "clocks": clk.summary(),
+        "timed_as": "eager steps, CUDA events around each step",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    mdist.shutdown()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -518,6 +584,8 @@ def main():
     ap.add_argument("--no-companions", action="store_true",
                     help="skip the attention timing of the other target workloads")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of as a graph")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: time the step over the cache quantized to FP8 E4M3 (CUDA-core kernels)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -525,6 +593,8 @@ def main():
     w = synth.workload(int(name) if name.isdigit() else name)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.cache == "fp8":
+        return run_fp8(args, w)
     return run_ours(args, w)
 
 

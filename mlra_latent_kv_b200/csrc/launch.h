@@ -41,13 +41,6 @@ cudaError_t launch_absorb(int dtype, bool q_bf16, const void* q_nope, const void
 cudaError_t launch_attend_simt(int dtype, const float* q_ws, const void* lat, const void* rop, const int* page_table,
                                const int* seq_lens, float* o_part, float* ml_part, int* err, const AttnArgs& a,
                                cudaStream_t st);
-// FP8 cache (E4M3 codes, fp32 scale per page and tensor): the CUDA-core attention
-// over it, and the quantizer of a bf16 (dtype 1) or fp32 pool.
-cudaError_t launch_attend_simt_fp8(const float* q_ws, const uint8_t* lat, const uint8_t* rop, const float* lat_scale,
-                                   const float* rop_scale, const int* page_table, const int* seq_lens, float* o_part,
-                                   float* ml_part, int* err, const AttnArgs& a, cudaStream_t st);
-cudaError_t launch_quantize_pages(int dtype, const void* pool, int num_pages, int n_per_page, uint8_t* codes,
-                                  float* scales, cudaStream_t st);
 cudaError_t launch_combine(bool out_bf16, const float* o_part, const float* ml_part, const int* seq_lens,
                            void* o_lat, const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_upproj(int dtype, bool in_bf16, const void* o_lat, const void* W_UV, void* out, const UpArgs& a,

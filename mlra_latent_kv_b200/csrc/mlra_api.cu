@@ -6,6 +6,7 @@
 #include <cstring>
 #include <string>
 
+#include "fp8_cache.h"
 #include "../../include/mlra.h"
 #include "attn_tc.h"
 #include "gemm_tc.h"

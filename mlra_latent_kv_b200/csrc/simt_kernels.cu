@@ -5,6 +5,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "fp8_cache.h"
 #include "launch.h"
 
 namespace mlra {
