@@ -16,6 +16,7 @@ from _support import compare, oracle_inputs, rel_l2
 pytestmark = pytest.mark.gpu
 
 CASES = {
+    "tiny_mla_fp32": dict(),
     "paged_varlen_h32": dict(B=3, seq_len_range=(1, 700)),
     "dsv2_contiguous": dict(B=2, seq_len=300),
     "mlra4": dict(B=2, seq_len=333),
@@ -40,7 +41,7 @@ def test_quantizer_matches_the_oracle_codec(name):
         np.testing.assert_array_equal(scales.cpu().numpy(), ref_scales)
         got = codes.cpu().numpy()
         nan = np.isnan(x)
-        assert nan.any()                                   # the unused slots are poisoned
+        assert nan.any() or name == "tiny_mla_fp32"       # the unused slots are poisoned (the tiny pool is full)
         np.testing.assert_array_equal(got[~nan], ref_codes[~nan])
         assert np.all(np.isnan(fp8.e4m3_decode(got[nan])))
 
