@@ -125,12 +125,16 @@ ATTN_SOURCES = ("attn_tc.cu", "attn_small.cu", "attn_branch.cu", "attn_common.cu
 
 
 def source_digest() -> str:
-    """Digest of the sources the attention kernel is built from (a stored ncu
-    traffic figure is used only while it matches)."""
+    """Digest of the code the attention kernel is built from, with `//`
+    comments and blank lines left out (a stored ncu traffic figure is used
+    only while it matches; a comment does not change the kernel)."""
     h = hashlib.sha256()
     for name in ATTN_SOURCES:
-        with open(os.path.join(ROOT, "mlra_latent_kv_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "mlra_latent_kv_b200", "csrc", name), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode("utf-8") + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -31,9 +31,15 @@
 //     (A = P in TMEM, B = the unit's latent read MN-major, N = 128 dims) are
 //     issued by two warps.
 //   * Softmax: per TMEM lane quarter, four warps, one per 32 tokens of the
-//     unit; they agree on the unit's row maximum through shared memory.  O is
-//     rescaled only when the running max grows by more than 2^8.  The first
-//     warp of each quarter also loads the query rows per piece.
+//     unit; they agree on the unit's row maximum through shared memory.  Past
+//     a piece's first unit each warp exponentiates against the running max
+//     while that exchange is in flight (capped so nothing overflows) and
+//     corrects afterwards when the unit's maximum jumped, so the exchange is
+//     off the critical path.  O is rescaled only when the running max grows by
+//     more than 2^8.  The first warp of each quarter also loads the query rows
+//     per piece.
+//   * Producer: the whole TMA warp walks the pages; per unit, lanes fetch the
+//     look-ahead page ids and issue the unit's six tile loads at once.
 //   * Rows past the sequence end in the last page are zeroed in shared memory
 //     before the MMAs read them (a NaN there would poison P.V even at P = 0).
 //   * Every wait is bounded; a wait that runs out sets the CTA's abort flag and
