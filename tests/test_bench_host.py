@@ -56,8 +56,10 @@ def test_source_digest_follows_every_attention_source(tmp_path, monkeypatch):
     for name in bench.ATTN_SOURCES:
         p = csrc / name
         orig = p.read_bytes()
-        p.write_bytes(orig + b"\n")
+        p.write_bytes(orig + b"\nconstexpr int kNotThere = 1;\n")
         assert bench.source_digest() != base, f"{name} is not covered by the digest"
+        p.write_bytes(orig + b"\n// a comment changes no kernel\n\n")
+        assert bench.source_digest() == base, f"a comment in {name} changed the digest"
         p.write_bytes(orig)
     assert bench.source_digest() == base
 
