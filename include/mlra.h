@@ -292,11 +292,16 @@ MLRA_API mlra_status latent_store(const mlra_dims* dims, int n_tokens, const voi
  * MLRA_NOALLOC_SCRATCH_BYTES (4 MiB), which every GPU that loads the library
  * holds until the process exits.  There is no counterpart on the pages; this
  * is an interface convenience only.
- *   - Scratch needed: ceil(d_model/64) * B * (d_c + d_r) * 4 bytes; a call
- *     that needs more returns MLRA_ERR_UNSUPPORTED and enqueues nothing.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.  The address is kept per device and
+ *   - Scratch needed: none when the columns split into 16-byte groups (d_r
+ *     a multiple of 8 for bf16, of 4 for fp32; d_c always is) and d_model <=
+ *     81920: that append is one launch whose partial sums stay on chip (and
+ *     latent_append_workspace_bytes is then the 256-byte error record).
+ *     Otherwise the two-kernel form needs ceil(d_model/64) * B * (d_c + d_r)
+ *     * 4 bytes; a call that needs more than the scratch returns
+ *     MLRA_ERR_UNSUPPORTED and enqueues nothing.
+ *   - The first call on each device that uses the scratch looks up the
+ *     array's device address (cudaGetSymbolAddress) with that device
+ *     current; make that first call before any stream capture.  The address is kept per device and
  *     context; after cudaDeviceReset (or any release of a device's primary
  *     context) call mlra_shutdown() before the next call, which forgets it.
  *   - Memory: the array lives in the same device module as every kernel of

@@ -2,8 +2,11 @@
 // device memory (an engine whose cache pool owns all HBM and forbids later
 // cudaMalloc, a decode loop that must not risk the synchronisation an
 // allocation can cause, a plugin host that passes buffers but no allocator).
-// The split-K partial sums that latent_append keeps in the caller's workspace
-// live here in one fixed, file-scope device array instead.  There is no
+// The one-launch append keeps its partial sums on chip and needs no scratch;
+// the two-kernel form (columns that do not split into 16-byte groups, or a
+// hidden width too large for the one-launch form's shared memory) keeps its
+// split-K partial sums here, in one fixed, file-scope device array, where
+// latent_append keeps them in the caller's workspace.  There is no
 // counterpart on the pages.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -11,6 +14,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "append_forms.h"
 #include "launch.h"
 
 using namespace mlra;
@@ -101,7 +105,8 @@ extern "C" MLRA_API mlra_status latent_append_noalloc(const mlra_dims* dims, int
   }
   if (pos == nullptr || page_table == nullptr) return internal_fail(MLRA_ERR_INVALID_ARG, "pos/page_table is NULL");
   const int KS = (d_model + 63) / 64;
-  const size_t need = (size_t)KS * dims->B * (dims->d_c + dims->d_r) * sizeof(float);
+  const bool scratch_used = append_uses_scratch(dims->dtype, d_model, dims->d_c, dims->d_r);
+  const size_t need = scratch_used ? (size_t)KS * dims->B * (dims->d_c + dims->d_r) * sizeof(float) : 0;
   if (need > MLRA_NOALLOC_SCRATCH_BYTES) {
     snprintf(msg, sizeof(msg),
              "latent_append_noalloc: B=%d, d_model=%d, d_c+d_r=%d need %zu bytes of scratch; the fixed scratch "
@@ -110,12 +115,15 @@ extern "C" MLRA_API mlra_status latent_append_noalloc(const mlra_dims* dims, int
     return internal_fail(MLRA_ERR_UNSUPPORTED, msg);
   }
   void* scratch = nullptr;
-  cudaError_t e = scratch_address(&scratch);
-  if (e != cudaSuccess) {
-    snprintf(msg, sizeof(msg), "latent_append_noalloc: looking up the scratch address: %s", cudaGetErrorString(e));
-    return internal_fail(MLRA_ERR_CUDA, msg);
+  cudaError_t e = cudaSuccess;
+  if (scratch_used) {
+    e = scratch_address(&scratch);
+    if (e != cudaSuccess) {
+      snprintf(msg, sizeof(msg), "latent_append_noalloc: looking up the scratch address: %s", cudaGetErrorString(e));
+      return internal_fail(MLRA_ERR_CUDA, msg);
+    }
   }
-  // pass 1 writes every partial sum pass 2 reads, so the scratch needs no clearing
+  // the two-kernel form's pass 1 writes every partial sum pass 2 reads, so the scratch needs no clearing
   AppendArgs a{dims->B, d_model, dims->d_c, dims->d_r, dims->max_pages_per_seq, dims->num_pages, KS};
   e = launch_append(dims->dtype, h, W_DKV, W_KR, pos, page_table, latent_cache, rope_cache,
                     static_cast<float*>(scratch), /*err=*/nullptr, a, internal_rope_table(dims), stream);

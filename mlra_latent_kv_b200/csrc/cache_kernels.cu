@@ -8,13 +8,17 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "host_cache.h"
+#include "append_forms.h"
 #include "launch.h"
 #include "ptx.cuh"
 
 namespace mlra {
 
 // ---------------------------------------------------------------------------
-// latent_append, pass 1: split-K partial products
+// latent_append, two-kernel form (the shapes the one-launch form below does
+// not take: columns that do not split into 16-byte groups, or a hidden width
+// whose chunk outgrows its shared memory), pass 1: split-K partial products
 //   part[ks, b, j] = sum_{k in chunk ks} h[b, k] * Wcat[k, j],   Wcat = [W_DKV | W_KR]
 // grid (KS) chunks of 64 weight rows.  A thread owns kCG adjacent columns (one
 // 16-byte load per weight row) in one of kRG row groups (rows rg, rg + kRG,
@@ -184,6 +188,171 @@ __global__ void append_finalize_kernel(const float* __restrict__ part, const int
   }
 }
 
+// ---------------------------------------------------------------------------
+// latent_append in one launch, for 16-byte column groups (d_r a multiple of
+// 16 / sizeof(T)): one cluster of kApSplit CTAs per block of kApCols columns
+// of Wcat = [W_DKV | W_KR].  Rank r of the cluster reads rows [r rc, r rc + rc)
+// of its columns (rc = ceil(D / kApSplit)) exactly once, every thread with all
+// of its row loads in flight at once; the CTA adds its row groups in a fixed
+// order through shared memory and stores its kApCols x kAppendB sums into rank
+// 0's shared memory; after the cluster barrier rank 0 adds the ranks' sums in
+// rank order, rotates the RoPE pairs at pos[b], rounds once and stores the
+// slot.  The partial sums never leave the chip, so this form needs no scratch,
+// and the sum has the same order on every call.
+// ---------------------------------------------------------------------------
+constexpr int kApCols = 32;     // columns per cluster (d_c is a multiple of 32: a block is latent or rope)
+constexpr int kApSplit = 8;     // CTAs per cluster: row chunks of the hidden dim
+constexpr int kApThreads = 256;
+constexpr int kApLoads = 10;    // row loads of a thread in flight at once (all of them at d_model = 5120)
+constexpr int kApOut = kApCols * kAppendB;  // a CTA's sums: [sequence][column]
+constexpr int kApRedStride = kApOut + 1;    // a row group's sums; the odd stride keeps the stores conflict-free
+constexpr size_t kApMaxDynSmem = 160 * 1024;  // hs: kAppendB x rc floats
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t caddr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
+}
+
+template <typename T>
+__global__ void __cluster_dims__(1, kApSplit, 1) __launch_bounds__(kApThreads, 2)
+    append_cluster_kernel(const T* __restrict__ h, const T* __restrict__ W_DKV, const T* __restrict__ W_KR,
+                          const int* __restrict__ pos, const int* __restrict__ page_table, T* __restrict__ lat,
+                          T* __restrict__ rop, int* __restrict__ err, AppendArgs a, RopeTable tab) {
+  constexpr int kCG = 16 / (int)sizeof(T);   // columns of one 16-byte load
+  constexpr int kNCG = kApCols / kCG;        // column groups
+  constexpr int kRG = kApThreads / kNCG;     // row groups
+  __shared__ float red[kRG][kApRedStride];
+  __shared__ float gath[kApSplit][kApOut];   // used in rank 0: every rank's sums
+  extern __shared__ float hs[];              // [kAppendB][rc]
+  const int W = a.d_c + a.d_r;
+  const int rc = (a.D + kApSplit - 1) / kApSplit;
+  const int rank = (int)ptx::cluster_ctarank();
+  const int k0 = rank * rc;
+  const int nk = max(0, min(rc, a.D - k0));
+  const int cg = threadIdx.x % kNCG, rg = threadIdx.x / kNCG;
+  const int j = blockIdx.x * kApCols + cg * kCG;
+  const bool col_ok = j < W;
+  const T* wp = !col_ok ? W_KR : j < a.d_c ? W_DKV + j : W_KR + (j - a.d_c);  // never read when !col_ok
+  const int ld = j < a.d_c ? a.d_c : a.d_r;
+  const uint32_t to_rank0 = ptx::map_to_cta(ptx::smem_u32(&gath[rank][0]), 0);
+  // every CTA of the cluster must have started before rank 0's shared memory is written: arrive now, wait
+  // just before the first remote store
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  bool first = true;
+  for (int b0 = 0; b0 < a.B; b0 += kAppendB) {
+    // rank 0's storing threads: thread t < kApOut / 2 stores columns (jj, jj + 1) of sequence
+    // b0 + t / (kApCols / 2).  Its position is loaded now and its page id once the h rows are staged, so
+    // neither lookup delays the weight loads; both have landed by the time they are used.
+    const int pc = 2 * (threadIdx.x % (kApCols / 2)), si = threadIdx.x / (kApCols / 2);
+    const int jj = blockIdx.x * kApCols + pc;
+    const bool storer = rank == 0 && threadIdx.x < kApOut / 2 && b0 + si < a.B && jj < W;
+    const int p = storer ? __ldg(pos + b0 + si) : 0;
+    const bool pos_ok = p >= 0 && p < a.maxp * kPage;
+    int pg = -1;
+    float acc[kCG][kAppendB];
+#pragma unroll
+    for (int c = 0; c < kCG; ++c)
+#pragma unroll
+      for (int i = 0; i < kAppendB; ++i) acc[c][i] = 0.f;
+#pragma unroll 1
+    for (int r0 = rg; r0 < nk || r0 == rg; r0 += kRG * kApLoads) {
+      uint4 wv[kApLoads];
+#pragma unroll
+      for (int u = 0; u < kApLoads; ++u) {
+        const int k = r0 + u * kRG;
+        if (col_ok && k < nk) wv[u] = __ldg(reinterpret_cast<const uint4*>(wp + (size_t)(k0 + k) * ld));
+      }
+      if (r0 == rg) {  // the batch's h rows are staged while the first weight rows are in flight
+        // kApLoads values per thread in flight at once (all of them at d_model = 5120)
+        for (int e0 = threadIdx.x; e0 < kAppendB * rc; e0 += kApThreads * kApLoads) {
+          float v[kApLoads];
+#pragma unroll
+          for (int u = 0; u < kApLoads; ++u) {
+            const int e = e0 + u * kApThreads, bi = e / rc, k = e % rc;
+            v[u] = (e < kAppendB * rc && k < nk && b0 + bi < a.B) ? to_f(h[(size_t)(b0 + bi) * a.D + k0 + k]) : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < kApLoads; ++u)
+            if (e0 + u * kApThreads < kAppendB * rc) hs[e0 + u * kApThreads] = v[u];
+        }
+        if (storer && pos_ok) pg = __ldg(page_table + (size_t)(b0 + si) * a.maxp + p / kPage);
+        __syncthreads();
+      }
+#pragma unroll
+      for (int u = 0; u < kApLoads; ++u) {
+        const int k = r0 + u * kRG;
+        if (col_ok && k < nk) {
+          const T* w = reinterpret_cast<const T*>(&wv[u]);
+#pragma unroll
+          for (int c = 0; c < kCG; ++c) {
+            const float wc = to_f(w[c]);
+#pragma unroll
+            for (int i = 0; i < kAppendB; ++i) acc[c][i] = fmaf(hs[i * rc + k], wc, acc[c][i]);
+          }
+        }
+      }
+    }
+    float sn = 0.f, cs = 1.f;
+    if (storer && pos_ok && jj >= a.d_c) rope_sincos(tab, (jj - a.d_c) / 2, p, &sn, &cs);
+#pragma unroll
+    for (int c = 0; c < kCG; ++c)
+#pragma unroll
+      for (int i = 0; i < kAppendB; ++i) red[rg][i * kApCols + cg * kCG + c] = acc[c][i];
+    __syncthreads();
+    float sum = 0.f;
+    if (threadIdx.x < kApOut)  // row groups in order
+      for (int g = 0; g < kRG; ++g) sum += red[g][threadIdx.x];
+    if (first) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    first = false;
+    if (threadIdx.x < kApOut) st_cluster_f32(to_rank0 + 4u * threadIdx.x, sum);  // into rank 0
+    ptx::cluster_sync();  // rank 0 now holds every rank's sums
+    // a position or page id out of range is reported and nothing is written for that sequence
+    bool write = false;
+    if (storer && !pos_ok) {
+      report_error(err, kErrDeviceCheck, b0 + si, p);
+    } else if (storer && (pg < 0 || pg >= a.num_pages)) {
+      report_error(err, kErrDeviceCheck, b0 + si, p);
+    } else {
+      write = storer;
+    }
+    if (write) {
+      const size_t slot = (size_t)pg * kPage + (p % kPage);
+      float x0 = 0.f, x1 = 0.f;
+      for (int q = 0; q < kApSplit; ++q) {  // ranks in order
+        x0 += gath[q][si * kApCols + pc];
+        x1 += gath[q][si * kApCols + pc + 1];
+      }
+      if (jj < a.d_c) {
+        lat[slot * a.d_c + jj] = from_f<T>(x0);
+        lat[slot * a.d_c + jj + 1] = from_f<T>(x1);
+      } else {
+        const int ir = (jj - a.d_c) / 2;
+        rop[slot * a.d_r + 2 * ir] = from_f<T>(x0 * cs - x1 * sn);
+        rop[slot * a.d_r + 2 * ir + 1] = from_f<T>(x0 * sn + x1 * cs);
+      }
+    }
+    if (b0 + kAppendB < a.B) ptx::cluster_sync();  // rank 0 has read its sums before the next batch rewrites them
+  }
+}
+
+template <typename T>
+static size_t append_cluster_dyn_smem(const AppendArgs& a) {
+  return sizeof(float) * kAppendB * (size_t)((a.D + kApSplit - 1) / kApSplit);
+}
+
+template <typename T>
+static cudaError_t launch_append_cluster(const void* h, const void* W_DKV, const void* W_KR, const int* pos,
+                                         const int* page_table, void* lat, void* rop, int* err, const AppendArgs& a,
+                                         const RopeTable& tab, cudaStream_t st) {
+  const size_t dyn = append_cluster_dyn_smem<T>(a);
+  auto k = append_cluster_kernel<T>;
+  const cudaError_t e = ensure_smem(reinterpret_cast<const void*>(k), (int)dyn);
+  if (e != cudaSuccess) return e;
+  const int n_cb = (a.d_c + a.d_r + kApCols - 1) / kApCols;
+  k<<<dim3(n_cb, kApSplit), kApThreads, dyn, st>>>((const T*)h, (const T*)W_DKV, (const T*)W_KR, pos, page_table,
+                                                   (T*)lat, (T*)rop, err, a, tab);
+  return cudaGetLastError();
+}
+
 template <typename T, int kCG>
 static cudaError_t launch_append_t(const void* h, const void* W_DKV, const void* W_KR, const int* pos,
                                    const int* page_table, void* lat, void* rop, float* part, int* err,
@@ -216,10 +385,22 @@ static cudaError_t launch_append_t(const void* h, const void* W_DKV, const void*
                             err, a, tab);
 }
 
+bool append_uses_scratch(int dtype, int D, int d_c, int d_r) {
+  const int cg = dtype == 1 ? 8 : 4;  // columns of a 16-byte load
+  const size_t dyn = sizeof(float) * kAppendB * (size_t)((D + kApSplit - 1) / kApSplit);
+  return d_c % cg != 0 || d_r % cg != 0 || dyn > kApMaxDynSmem;
+}
+
 cudaError_t launch_append(int dtype, const void* h, const void* W_DKV, const void* W_KR, const int* pos,
                           const int* page_table, void* lat, void* rop, float* part, int* err, const AppendArgs& a,
                           const RopeTable& tab, cudaStream_t st) {
-  // 16-byte weight loads when both blocks split into whole 16-byte groups, else 4-byte pairs
+  // one cluster-reduced launch where the columns split into 16-byte groups and the hidden chunk fits shared
+  // memory; else the split-K pair of kernels, whose partial sums go through `part`
+  if (!append_uses_scratch(dtype, a.D, a.d_c, a.d_r)) {
+    if (dtype == 1)
+      return launch_append_cluster<__nv_bfloat16>(h, W_DKV, W_KR, pos, page_table, lat, rop, err, a, tab, st);
+    return launch_append_cluster<float>(h, W_DKV, W_KR, pos, page_table, lat, rop, err, a, tab, st);
+  }
   if (dtype == 1) {
     if (a.d_c % 8 == 0 && a.d_r % 8 == 0)
       return launch_append_t<__nv_bfloat16, 8>(h, W_DKV, W_KR, pos, page_table, lat, rop, part, err, a, tab, st);

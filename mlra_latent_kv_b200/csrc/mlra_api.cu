@@ -11,6 +11,7 @@
 #include "attn_tc.h"
 #include "gemm_tc.h"
 #include "host_cache.h"
+#include "append_forms.h"
 #include "launch.h"
 
 using namespace mlra;
@@ -456,6 +457,7 @@ size_t latent_append_workspace_bytes(const mlra_dims* dims, int d_model) {
     fail(MLRA_ERR_INVALID_ARG, "d_model must be >= 1");
     return 0;
   }
+  if (!append_uses_scratch(dims->dtype, d_model, dims->d_c, dims->d_r)) return kErrBytes;  // the error record only
   const int KS = (d_model + 63) / 64;
   return kErrBytes + round_up((size_t)KS * dims->B * (dims->d_c + dims->d_r) * 4, 256);
 }

@@ -132,10 +132,22 @@ def test_tc_request_outside_tc_shapes_is_unsupported(L):
 def test_append_and_store_validation(L):
     d = _dims()
     assert L.latent_append_workspace_bytes(ctypes.byref(d), 0) == 0
+    # 16-byte column groups: the one-launch form keeps its sums on chip, only the error record
     n = L.latent_append_workspace_bytes(ctypes.byref(d), 5120)
-    assert n == 256 + (80 * 4 * 576 * 4 + 255) // 256 * 256
+    assert n == 256
     st = L.latent_append(ctypes.byref(d), 5120, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n - 1, None)
     assert st == 3
+    # d_r = 62 does not split into 16-byte groups: the two-kernel form's split-K sums, 80 chunks of 64 rows
+    d62 = _dims(d_r=62)
+    n62 = L.latent_append_workspace_bytes(ctypes.byref(d62), 5120)
+    assert n62 == 256 + (80 * 4 * 574 * 4 + 255) // 256 * 256
+    assert L.latent_append(ctypes.byref(d62), 5120, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, n62 - 1,
+                           None) == 3
+    # fp32 groups are 4 columns wide: d_r = 60 still takes the one-launch form
+    assert L.latent_append_workspace_bytes(ctypes.byref(_dims(d_r=60, dtype="f32")), 5120) == 256
+    # a hidden width whose chunk (kAppendB rows of ceil(d_model / 8) floats) outgrows shared memory: two kernels
+    big = 8 * 10240 + 8
+    assert L.latent_append_workspace_bytes(ctypes.byref(d), big) == 256 + ((big + 63) // 64 * 4 * 576 * 4 + 255) // 256 * 256
     st = L.latent_store(ctypes.byref(d), -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None)
     assert st == 1
     st = L.latent_store(ctypes.byref(d), 10, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 256, None)

@@ -48,7 +48,9 @@ def test_noalloc_matches_latent_append_on_two_calls():
 
 def test_noalloc_refuses_more_than_its_scratch():
     s = _session(23, 2, (64, 64))
-    big = abi.make_dims(B=64, H=s.w.H, d_h=s.w.d_h, d_v=s.w.d_v, d_c=s.w.d_c, d_r=s.w.d_r,
+    # d_r = 62 does not split into 16-byte column groups: the two-kernel form, whose split-K sums
+    # (80 chunks x 64 sequences x 574 columns of fp32) outgrow the fixed scratch
+    big = abi.make_dims(B=64, H=s.w.H, d_h=s.w.d_h, d_v=s.w.d_v, d_c=s.w.d_c, d_r=62,
                         max_pages_per_seq=s.maxp, num_pages=s.num_pages)
     before = s.latent_cache.clone()
     with pytest.raises(abi.MlraError) as ei:
