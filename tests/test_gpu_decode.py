@@ -235,22 +235,39 @@ def test_device_check_bad_page_id(kernel):
     s.check()  # cleared
 
 
-FULL_PAIRS = {
+# Sampled (b, h) rows at full size: sequences spread over the batch plus the longest and the shortest, heads
+# spread over all four TMEM lane quarters; (sequences, heads) per workload, sized so the fp64 oracle takes seconds.
+FULL_SAMPLE = {
     "tiny_mla_fp32": None,
-    "dsv2_contiguous": [(0, 0), (5, 77), (31, 127), (17, 3)],
-    "paged_varlen_h32": [(0, 0), (13, 31), (40, 7), (63, 16)],
-    "mlra4": [(0, 0), (11, 64), (31, 127)],
-    "longctx_append": [(0, 0), (3, 127), (1, 50)],
+    "dsv2_contiguous": (8, 8),
+    "paged_varlen_h32": (8, 5),
+    "mlra4": (6, 6),
+    "longctx_append": (4, 5),
 }
 
 
-@pytest.mark.parametrize("name", list(FULL_PAIRS))
+def full_pairs(name, w, inp):
+    if FULL_SAMPLE[name] is None:
+        return None
+    nb, nh = FULL_SAMPLE[name]
+    lens = inp["attn_lens"].numpy()
+    bs = set(np.linspace(0, w.B - 1, nb).round().astype(int).tolist())
+    bs |= {int(lens.argmax()), int(lens.argmin())}
+    hs = sorted(set(np.linspace(0, w.H - 1, nh).round().astype(int).tolist()))
+    return [(b, h) for b in sorted(bs) for h in hs]
+
+
+@pytest.mark.parametrize("name", list(FULL_SAMPLE))
 def test_full_size_sampled(name):
     """Full workload sizes, default launch configuration (the one the benchmark times)."""
     w = synth.workload(name)
-    err, tol, out, ref, _ = run_case(w, "auto", pairs=FULL_PAIRS[name])
+    inp = synth.make_inputs(w)
+    pairs = full_pairs(name, w, inp)
+    err, tol, out, ref, _ = run_case(w, "auto", pairs=pairs, inp=inp)
     assert err <= tol, f"{name}: {err:.3e} > {tol:.3e}"
     assert torch.isfinite(out.float()).all()
+    if pairs is not None:
+        assert len(ref) == len(pairs) >= 12
 
 
 @pytest.mark.parametrize("name", ["dsv2_contiguous", "mlra4"])
