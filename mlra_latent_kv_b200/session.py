@@ -137,10 +137,18 @@ class DecodeSession:
         if self.appends:
             abi.check_status(self.app_ws)
 
+    def append_kernels(self) -> int:
+        """Kernels one latent_append launches: one for the one-launch form,
+        whose workspace is the 256-byte error record alone, two for the
+        two-kernel form (partial sums in the workspace, then the finalize)."""
+        if not self.appends:
+            return 0
+        return 1 if abi.append_workspace_bytes(self.dims, self.d_model) == 256 else 2
+
     def kernels_per_step(self) -> int:
-        """Kernels one step launches: append (2, when it appends) plus the
+        """Kernels one step launches: the append's (when it appends) plus the
         decode call's own launches, as the library plans them."""
-        return (2 if self.appends else 0) + abi.describe_plan(self.dims)["kernels"]
+        return self.append_kernels() + abi.describe_plan(self.dims)["kernels"]
 
     def plan(self) -> dict:
         """The decode call's kernel plan (family and per-stage kernel names)."""

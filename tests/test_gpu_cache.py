@@ -93,6 +93,7 @@ def test_latent_append_values_and_addressing(name, over):
     # the workspace the session sized: the error record alone for the one-launch form
     one_launch = (w.d_r % (8 if w.dtype == "bf16" else 4) == 0) and w.append_d_model <= 8 * 10240
     assert (abi.append_workspace_bytes(s.dims, s.d_model) == 256) == one_launch
+    assert s.append_kernels() == (1 if one_launch else 2)
 
 
 def test_latent_append_rejects_position_outside_table():
